@@ -1,0 +1,654 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 E4M3 quantization hot path on B200.
+
+One step is one 4593-token prefill through every operation of the path:
+  * fp8_group_quant of the 4593 x 5120 bf16 activation (1x128 groups);
+  * for each of 16 layers (4 KV heads x 128 dims, 8192-block pools of 16
+    slots), the calibrating KV write of that layer's 4593 tokens, arriving in
+    two chunks: 4095 tokens inside the window (one fused pass: absmax, staging
+    copy, provisional-scale write), then 498 tokens that reach the 4096-token
+    window (absmax; freeze and replay of the 4095 staged tokens; write of the
+    crossing chunk at the frozen scale).
+That is 1 + 16 x 4 = 65 kernel launches, issued through the C ABI and
+replayed as one CUDA graph.  Before every step L2 is flushed (a 2x-L2 write)
+and the calibrators' device state is reset, both outside the timed region.
+
+`value` is effective HBM GB/s: the algorithmic bytes of the step (each
+kernel's compulsory reads and writes) divided by the step time measured with
+CUDA events.  Per-kernel times come from event nodes between the launches.
+`--impl reference` times the CPU oracle on a bounded sample of the same step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "FP8 quant/KV-write effective HBM GB/s and % of B200 peak; tokens/s"
+TOKENS = workloads.LARGE_TOKENS          # 4593
+CHUNK1, CHUNK2 = workloads.LARGE_CHUNKS  # 4095, 498
+E = workloads.KV_HEADS * workloads.HEAD_DIM
+M, K = workloads.PREFILL_M, workloads.PREFILL_K
+
+# Algorithmic bytes per launch (compulsory reads + writes of each kernel).
+PER_TOKEN = {
+    "observe_stage_write": 2 * E * 2 + 8 + 2 * E + 2 * E * 2 + 8,   # 5136
+    "amax": 2 * E * 2,                                             # 2048
+    "freeze_replay": 2 * E * 2 + 8 + 2 * E,                        # 3080
+    "kv_write": 2 * E * 2 + 8 + 2 * E,                             # 3080
+}
+GROUP_QUANT_BYTES = M * K * 3 + M * (K // 128) * 4                 # 71,283,360
+
+
+def launch_bytes(label: str) -> int:
+    if label == "group_quant":
+        return GROUP_QUANT_BYTES
+    tokens = {"observe_stage_write": CHUNK1, "amax": CHUNK2, "freeze_replay": CHUNK1,
+              "kv_write": CHUNK2}[label]
+    return PER_TOKEN[label] * tokens
+
+
+def step_bytes(layers: int) -> int:
+    per_layer = sum(launch_bytes(k) for k in ("observe_stage_write", "amax", "freeze_replay",
+                                              "kv_write"))
+    return GROUP_QUANT_BYTES + layers * per_layer
+
+
+# ---------------------------------------------------------------------------
+# process group plumbing (one process per GPU; no data-path collective)
+
+
+class Dist:
+    def __init__(self) -> None:
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend: str, timeout_s: float = 120.0) -> None:
+        if self.world > 1 and not torch.distributed.is_initialized():
+            import datetime
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            kw = {}
+            if backend == "nccl":
+                kw["device_id"] = torch.device("cuda", self.local_rank)
+            torch.distributed.init_process_group(
+                backend, rank=self.rank, world_size=self.world,
+                timeout=datetime.timedelta(seconds=timeout_s), **kw)
+            self.pg = True
+
+    def barrier(self) -> None:
+        if self.pg:
+            torch.distributed.barrier()
+
+    def reduce(self, value: float, op: str, device) -> float:
+        if not self.pg:
+            return value
+        t = torch.tensor([value], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(
+            t, op=torch.distributed.ReduceOp.MAX if op == "max" else torch.distributed.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self) -> None:
+        if self.pg:
+            torch.distributed.destroy_process_group()
+            self.pg = False
+
+
+def aggregate(dist: Dist, seconds: float, units: float, device) -> tuple[float, float]:
+    """Whole-job (max seconds over ranks, total units over ranks)."""
+    return dist.reduce(seconds, "max", device), dist.reduce(units, "sum", device)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+
+def smi_gpu_id(local_rank: int) -> str:
+    """nvidia-smi's id of this rank's GPU (CUDA_VISIBLE_DEVICES may remap)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    return ids[local_rank] if local_rank < len(ids) else str(local_rank)
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index: str) -> None:
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="fp8q_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"error": "nvidia-smi unavailable"}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"error": "no samples", "samples": 0}
+        reasons = sorted({self.REASONS[i] for _, _, flags in rows
+                          for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "window": "warm-up and timed steps"}
+
+
+# ---------------------------------------------------------------------------
+# the native step
+
+
+class Workload:
+    """Device-resident inputs, outputs, pools and calibrator state of one step."""
+
+    def __init__(self, device, layers: int) -> None:
+        import paged_kv_cache_group_b200 as fp8q
+        self.fp8q = fp8q
+        self.device = device
+        self.layers = layers
+        self.host_x = workloads.prefill_quant()
+        self.host_kv = [workloads.large_kv_layer(l) for l in range(layers)]
+        self.x = self._bf16(self.host_x)
+        self.q = torch.empty((M, K), dtype=torch.uint8, device=device)
+        self.s = torch.empty((M, K // 128), dtype=torch.float32, device=device)
+        shape = (workloads.LARGE_NUM_BLOCKS, 16, workloads.KV_HEADS, workloads.HEAD_DIM)
+        self.k, self.v, self.slots, self.k_pool, self.v_pool = [], [], [], [], []
+        for b in self.host_kv:
+            self.k.append(self._bf16(b.k).view(TOKENS, workloads.KV_HEADS, workloads.HEAD_DIM))
+            self.v.append(self._bf16(b.v).view(TOKENS, workloads.KV_HEADS, workloads.HEAD_DIM))
+            self.slots.append(torch.from_numpy(b.slot_mapping).to(device))
+            self.k_pool.append(torch.full(shape, workloads.SENTINEL, dtype=torch.uint8, device=device))
+            self.v_pool.append(torch.full(shape, workloads.SENTINEL, dtype=torch.uint8, device=device))
+        self.states = torch.zeros((layers, 4), dtype=torch.float32, device=device)
+        self.states_init = torch.tensor([0.0, 0.0, 2.0, 2.0], device=device).repeat(layers, 1)
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        self.flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+
+    def _bf16(self, bits):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+        return t.view(torch.bfloat16).to(self.device)
+
+    def calibrators(self):
+        fp8q = self.fp8q
+        return [fp8q.KvCalibration(workloads.LARGE_WINDOW_REQUEST, 1.0, workloads.KV_HEADS,
+                                   workloads.HEAD_DIM, self.device, state=self.states[l])
+                for l in range(self.layers)]
+
+    def reset(self, i: int) -> None:
+        self.states.copy_(self.states_init)
+        self.flush_buf.fill_(i & 0xFF)
+
+    def issue(self, calibs, mark) -> None:
+        fp8q = self.fp8q
+        fp8q.fp8_group_quant(self.x, self.q, self.s)
+        mark("group_quant")
+        for l, c in enumerate(calibs):
+            k, v, s = self.k[l], self.v[l], self.slots[l]
+            kp, vp = self.k_pool[l], self.v_pool[l]
+            st = c.observe_write(k[:CHUNK1], v[:CHUNK1], s[:CHUNK1], kp, vp)
+            assert st == fp8q.STEP_STAGE, st
+            mark("observe_stage_write")
+            st = c.observe(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:])
+            assert st == fp8q.STEP_FREEZE, st
+            mark("amax")
+            n = c.freeze_replay(kp, vp)
+            assert n == CHUNK1, n
+            mark("freeze_replay")
+            fp8q.fp8_kv_write(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:], kp, vp, scale_dev=c.scale_dev)
+            mark("kv_write")
+
+
+def labels_of(layers: int) -> list[str]:
+    return ["group_quant"] + ["observe_stage_write", "amax", "freeze_replay", "kv_write"] * layers
+
+
+def capture(w: Workload, stream, with_events: bool):
+    """Capture one step into a CUDA graph; event nodes between launches."""
+    labels = labels_of(w.layers)
+    events = [torch.cuda.Event(enable_timing=True, external=True)
+              for _ in range(len(labels) + 1)] if with_events else []
+    with torch.cuda.stream(stream):
+        calibs = w.calibrators()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    before = w.fp8q.launch_count()
+    pos = [0]
+
+    def mark(_label):
+        if with_events:
+            pos[0] += 1
+            events[pos[0]].record()
+
+    with torch.cuda.graph(graph, stream=stream):
+        if with_events:
+            events[0].record()
+        w.issue(calibs, mark)
+    launches = w.fp8q.launch_count() - before
+    # The graph writes into these calibrators' staging tensors on every
+    # replay: the caller keeps them alive as long as the graph.
+    return graph, events, labels, launches, calibs
+
+
+def run_native(args, dist: Dist) -> dict | None:
+    import paged_kv_cache_group_b200 as fp8q
+    torch.cuda.set_device(dist.local_rank)
+    device = torch.device("cuda", dist.local_rank)
+    dist.init("nccl")
+    w = Workload(device, args.layers)
+    stream = torch.cuda.Stream(device)
+
+    # eager warm-up: fills the library's launch-geometry caches, checks the flow
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            w.reset(i)
+            w.issue(w.calibrators(), lambda _l: None)
+    torch.cuda.synchronize()
+    assert fp8q.fp8q_device_error(clear=True) == 0
+
+    graph, events, labels, launches, graph_calibs = capture(w, stream, with_events=True)
+    assert launches == len(labels), (launches, len(labels))
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    clocks = ClockSampler(smi_gpu_id(dist.local_rank)) if dist.rank == 0 else None
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            w.reset(i)
+            graph.replay()
+    torch.cuda.synchronize()
+
+    dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, per_label = [], {l: [] for l in set(labels)}
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            w.reset(i)
+            start.record()
+            graph.replay()
+            end.record()
+            end.synchronize()
+            step_ms.append(start.elapsed_time(end))
+            for j, lab in enumerate(labels):
+                per_label[lab].append(events[j].elapsed_time(events[j + 1]))
+    torch.cuda.synchronize()
+    dist.barrier()
+    clock_info = clocks.stop() if clocks is not None else None
+    gpu_launches = launches * args.steps
+
+    total_s = sum(step_ms) / 1e3
+    bytes_rank = step_bytes(args.layers) * args.steps
+    max_s, total_bytes = aggregate(dist, total_s, bytes_rank, device)
+    tokens_total = dist.reduce(TOKENS * args.steps, "sum", device)
+
+    # correctness of the timed replays: the last step's pools and codes must be
+    # those of a fresh eager step (identical inputs, deterministic kernels)
+    q_graph = w.q.clone()
+    pools_graph = (w.k_pool[-1].clone(), w.v_pool[-1].clone())
+    with torch.cuda.stream(stream):
+        w.reset(0)
+        w.issue(w.calibrators(), lambda _l: None)
+    torch.cuda.synchronize()
+    assert torch.equal(q_graph, w.q)
+    assert torch.equal(pools_graph[0], w.k_pool[-1]) and torch.equal(pools_graph[1], w.v_pool[-1])
+    del pools_graph
+    assert fp8q.fp8q_device_error(clear=True) == 0
+
+    # eager (no graph) step time through the Python binding, for context
+    eager_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(min(args.steps, 20)):
+            calibs = w.calibrators()
+            w.reset(i)
+            start.record()
+            w.issue(calibs, lambda _l: None)
+            end.record()
+            end.synchronize()
+            eager_ms.append(start.elapsed_time(end))
+
+    targets = measure_targets(w, stream, args)
+    e2e = None if args.no_e2e else measure_e2e(w, stream, args)
+    del graph
+    for c in graph_calibs:
+        c.close()
+    peaks = measured_peaks()
+    result = None
+    if dist.rank == 0:
+        kernels = {}
+        for lab, ts in per_label.items():
+            n_per_step = labels.count(lab)
+            avg_us = 1e3 * sum(ts) / len(ts)
+            b = launch_bytes(lab)
+            gbs = b / (avg_us * 1e-6) / 1e9
+            kernels[lab] = {"launches_per_step": n_per_step, "avg_us": round(avg_us, 3),
+                            "bytes_per_launch": b, "gbs": round(gbs, 1),
+                            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                            "share_of_step": round(n_per_step * avg_us / (1e3 * statistics.mean(step_ms)), 4)}
+        dominant = max(kernels, key=lambda k: kernels[k]["launches_per_step"] * kernels[k]["avg_us"])
+        dk = kernels[dominant]
+        ms = 1e3 * max_s / args.steps
+        result = {
+            "metric": METRIC, "value": round(total_bytes / max_s / 1e9, 2), "unit": "GB/s",
+            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic: seeded Philox draws rounded to bf16 (no weights, no dataset)",
+            "config": {
+                "workload": (f"prefill of {TOKENS} tokens: group quant {M}x{K} bf16 + "
+                             f"{args.layers} layers x calibrating KV write "
+                             f"({workloads.KV_HEADS} KV heads x {workloads.HEAD_DIM}, "
+                             f"{workloads.LARGE_NUM_BLOCKS}-block pools of 16, window "
+                             f"{workloads.LARGE_WINDOW_REQUEST}->4096, chunks {CHUNK1}+{CHUNK2}: "
+                             "stage+write, freeze, replay, crossing write)"),
+                "l2": "flushed before every step (2x L2 write, untimed)",
+                "timing": "CUDA graph replay of the step's 65 launches; CUDA events",
+                "bytes_per_step": step_bytes(args.layers),
+                "parallelism": f"replicas x{dist.world} (one step per GPU, no collective)",
+            },
+            "tokens_per_s": round(tokens_total / max_s, 1),
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"],
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4),
+                         "traffic": committed_traffic(dominant),
+                         "peak_source": peaks["source"],
+                         "algorithmic_bytes_per_launch": dk["bytes_per_launch"]},
+            "kernels": kernels,
+            "targets": targets,
+            "eager_ms_per_step": round(statistics.median(eager_ms), 4),
+            "gpu_launches": gpu_launches,
+            "clocks": clock_info,
+        }
+        if e2e is not None:
+            result["e2e"] = e2e
+        if not args.no_cpu_baseline and dist.world == 1:
+            result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+    dist.close()
+    return result
+
+
+def measure_targets(w: Workload, stream, args) -> dict:
+    """The two stand-alone kernel figures the path is judged by: group quant of
+    the 4593 x 5120 activation, and the steady-state (post-freeze) KV write of
+    4593 tokens per layer, 16 layers back to back (one launch each)."""
+    fp8q = w.fp8q
+    peaks = measured_peaks()
+    out = {}
+    scale = torch.tensor([0.05, 0.05], dtype=torch.float32, device=w.device)
+    reps = max(3, min(args.steps, 50))
+
+    def timed(fn, n_launch):
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_launch + 1)]
+        with torch.cuda.stream(stream):
+            fn(lambda i: None)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            evs[0].record()
+            fn(lambda i: evs[i + 1].record())
+        times = []
+        with torch.cuda.stream(stream):
+            for i in range(reps):
+                w.flush_buf.fill_(i & 0xFF)
+                g.replay()
+                torch.cuda.synchronize()
+                times += [evs[j].elapsed_time(evs[j + 1]) for j in range(n_launch)]
+        del g
+        return statistics.mean(times) * 1e3
+
+    def gq(mark):
+        fp8q.fp8_group_quant(w.x, w.q, w.s)
+        mark(0)
+
+    us = timed(gq, 1)
+    gbs = GROUP_QUANT_BYTES / (us * 1e-6) / 1e9
+    out["group_quant_4593x5120"] = {"us": round(us, 3), "gbs": round(gbs, 1),
+                                    "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                    "tokens_per_s": round(M / (us * 1e-6), 1),
+                                    "vs_pages_h100_636_gbs": round(gbs / 636.0, 2)}
+
+    def kvw(mark):
+        for l in range(w.layers):
+            fp8q.fp8_kv_write(w.k[l], w.v[l], w.slots[l], w.k_pool[l], w.v_pool[l],
+                              scale_dev=scale)
+            mark(l)
+
+    us = timed(kvw, w.layers)
+    b = PER_TOKEN["kv_write"] * TOKENS
+    gbs = b / (us * 1e-6) / 1e9
+    out["kv_write_4593"] = {"us_per_layer": round(us, 3), "gbs": round(gbs, 1),
+                            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                            "tokens_per_s": round(TOKENS / (us * 1e-6), 1),
+                            "bytes_per_layer": b}
+    return out
+
+
+def measure_e2e(w: Workload, stream, args) -> dict:
+    """The same step through the public API with host inputs: every step copies
+    its inputs from pinned host memory and reads its results back."""
+    fp8q = w.fp8q
+    hx = torch.from_numpy(w.host_x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = [torch.from_numpy(b.k.view(np.int16)).view(torch.bfloat16).pin_memory() for b in w.host_kv]
+    hv = [torch.from_numpy(b.v.view(np.int16)).view(torch.bfloat16).pin_memory() for b in w.host_kv]
+    hs = [torch.from_numpy(b.slot_mapping).pin_memory() for b in w.host_kv]
+    oq = torch.empty((M, K), dtype=torch.uint8).pin_memory()
+    os_ = torch.empty((M, K // 128), dtype=torch.float32).pin_memory()
+    ost = torch.empty((w.layers, 4), dtype=torch.float32).pin_memory()
+    h2d = hx.numel() * 2 + sum(t.numel() * 2 for t in hk + hv) + sum(t.numel() * 8 for t in hs)
+    d2h = oq.numel() + os_.numel() * 4 + ost.numel() * 4
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    n = max(2, min(args.steps, 10))
+    with torch.cuda.stream(stream):
+        for i in range(n + 2):
+            calibs = w.calibrators()
+            w.reset(i)
+            start.record()
+            w.x.copy_(hx, non_blocking=True)
+            for l in range(w.layers):
+                w.k[l].view(TOKENS, E).copy_(hk[l], non_blocking=True)
+                w.v[l].view(TOKENS, E).copy_(hv[l], non_blocking=True)
+                w.slots[l].copy_(hs[l], non_blocking=True)
+            w.issue(calibs, lambda _l: None)
+            oq.copy_(w.q, non_blocking=True)
+            os_.copy_(w.s, non_blocking=True)
+            ost.copy_(w.states, non_blocking=True)
+            end.record()
+            end.synchronize()
+            if i >= 2:
+                times.append(start.elapsed_time(end))
+            for c in calibs:
+                c.close()
+    ms = statistics.mean(times)
+    assert fp8q.fp8q_device_error(clear=True) == 0
+    return {"value": round(step_bytes(w.layers) / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 4), "steps": n}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "measured (MEASURED_PEAKS.json hbm_gbs)"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "source": "fallback 6.65 TB/s"}
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_group_b200", "csrc", "*"))):
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(label: str):
+    """DRAM bytes per launch of `label` from the committed ncu summary, or None
+    when the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            t = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_hash") != source_hash():
+        return None
+    entry = t.get("kernels", {}).get(label)
+    return None if entry is None else entry.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (CPU baseline and the reference arm)
+
+SAMPLE_ROWS = 1148        # a quarter of the activation rows
+SAMPLE_LAYERS = 2         # two of the sixteen layers
+
+
+def reference_sample():
+    x = workloads.prefill_quant()[:SAMPLE_ROWS]
+    kv = [workloads.large_kv_layer(l) for l in range(SAMPLE_LAYERS)]
+    return x, kv
+
+
+def sample_bytes() -> int:
+    gq = SAMPLE_ROWS * K * 3 + SAMPLE_ROWS * (K // 128) * 4
+    per_layer = sum(launch_bytes(k) for k in ("observe_stage_write", "amax", "freeze_replay",
+                                              "kv_write"))
+    return gq + SAMPLE_LAYERS * per_layer
+
+
+def reference_step(x, kv) -> None:
+    import oracle
+    from oracle import calibration as cal
+    oracle.group_quant(x)
+    spec = workloads.large_kv_spec()
+    for b in kv:
+        c = cal.Fp8KvCalibration(0, workloads.LARGE_WINDOW_REQUEST, 1.0)
+        kp, vp = spec.new_pool().reshape(-1), spec.new_pool().reshape(-1)
+        chunks = [cal.KvBatch(p.k, p.v, p.slot_mapping, E, E)
+                  for p in workloads.split_batch(b, workloads.LARGE_CHUNKS)]
+        cal.run_calibrated_writes(c, chunks, workloads.KV_HEADS, workloads.HEAD_DIM, kp, vp, 16,
+                                  spec.cache_stride, spec.num_blocks)
+
+
+SAMPLE_DESC = (f"oracle (single-threaded C + Python calibration) on {SAMPLE_ROWS} of {M} "
+               f"activation rows and {SAMPLE_LAYERS} of 16 layers of the step; bytes counted "
+               "as for the GPU step")
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    x, kv = reference_sample()
+    reference_step(x, kv)                     # warm (builds and loads the oracle)
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 2:
+        t0 = time.perf_counter()
+        reference_step(x, kv)
+        times.append(time.perf_counter() - t0)
+    s = statistics.median(times)
+    return {"value": round(sample_bytes() / s / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "sample": SAMPLE_DESC, "repeats": len(times),
+            "host_cores": os.cpu_count()}
+
+
+def run_reference(args) -> dict | None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    x, kv = reference_sample()
+    for _ in range(args.warmup):
+        reference_step(x, kv)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        reference_step(x, kv)
+    s = (time.perf_counter() - t0) / args.steps
+    value = round(sample_bytes() / s / 1e9, 4)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(s * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: seeded Philox draws rounded to bf16 (no weights, no dataset)",
+        "config": {"workload": SAMPLE_DESC, "bytes_per_step": sample_bytes()},
+        "tokens_per_s": None,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": SAMPLE_DESC},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--layers", type=int, default=workloads.LARGE_LAYERS)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if a.steps < 1:
+        ap.error("--steps must be at least 1")
+    return a
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_native(args, Dist())
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,264 @@
+"""FP8 E4M3 quantization for B200: per-token 1x128-group activation
+quantization, the paged KV-cache quantize-and-scatter, and online calibration
+of the KV scales.
+
+The compute is the CUDA library libfp8q.so (C ABI: include/fp8q.h).  This
+module only marshals torch tensors (device memory) and streams into those
+calls; every step runs in the library's kernels.  Function names match the C
+ABI.  Importing fails if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import (CALIB_STATE_BYTES, DEVERR_BAD_SCALE, DEVERR_SLOT_OUT_OF_RANGE,  # noqa: F401
+                   MAX_STAGED_TOKENS, PROVISIONAL_SCALE, STEP_FREEZE, STEP_FROZEN, STEP_STAGE,
+                   STEP_STAGE_DECLINED, CalibStats, Fp8qError)
+
+lib = _abi.load()
+
+_BYTE_TYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _check(name: str, status: int) -> None:
+    if status != _abi.OK:
+        raise Fp8qError(name, status, lib.fp8q_status_string(status).decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _bf16_rows(t: torch.Tensor, name: str):
+    """[T, ...] bf16 with contiguous rows; returns (rows, row stride, E)."""
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+    rows = t.shape[0]
+    flat = t.reshape(rows, -1) if t.dim() > 2 else t
+    if flat.dim() != 2 or (flat.shape[1] > 1 and flat.stride(1) != 1):
+        raise ValueError(f"{name} rows must be contiguous")
+    if t.dim() > 2 and flat.data_ptr() != t.data_ptr():
+        raise ValueError(f"{name} rows must be contiguous")
+    return rows, flat.stride(0), flat.shape[1]
+
+
+# ---------------------------------------------------------------------------
+# activation quantization
+
+
+def fp8_group_quant(x: torch.Tensor, q: torch.Tensor | None = None,
+                    scales: torch.Tensor | None = None, stream=None):
+    """Quantize a bf16 ``[m, k]`` activation (k % 128 == 0, rows may be
+    strided) into E4M3 codes ``q [m, k]`` and fp32 ``scales [m, k/128]``."""
+    m, stride, k = _bf16_rows(x, "x")
+    if q is None:
+        q = torch.empty((m, k), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((m, k // 128), dtype=torch.float32, device=x.device)
+    if q.dtype not in _BYTE_TYPES or not q.is_contiguous() or q.numel() < m * k:
+        raise ValueError("q must be a contiguous uint8/float8_e4m3fn tensor of m*k elements")
+    if scales.dtype != torch.float32 or not scales.is_contiguous() or \
+            scales.numel() < m * (k // 128):
+        raise ValueError("scales must be a contiguous float32 tensor of m*(k/128) elements")
+    _check("fp8_group_quant", lib.fp8_group_quant(
+        _ptr(x), stride, _ptr(q), _ptr(scales), m, k, _stream(stream)))
+    return q, scales
+
+
+# ---------------------------------------------------------------------------
+# paged KV write
+
+
+def _pool_geometry(k_pool: torch.Tensor, v_pool: torch.Tensor, elems: int):
+    """Pools ``[num_blocks, block_size, heads, dim]`` (block stride may be padded)."""
+    for name, p in (("k_pool", k_pool), ("v_pool", v_pool)):
+        if p.dtype not in _BYTE_TYPES or not p.is_cuda:
+            raise TypeError(f"{name} must be a CUDA uint8/float8_e4m3fn tensor")
+    if k_pool.shape != v_pool.shape or k_pool.stride() != v_pool.stride():
+        raise ValueError("k_pool and v_pool must have the same shape and strides")
+    num_blocks, block_size = k_pool.shape[0], k_pool.shape[1]
+    inner = k_pool[0].numel() if num_blocks else block_size * elems
+    if inner != block_size * elems:
+        raise ValueError("pool block does not hold block_size * num_kv_heads * head_dim codes")
+    if num_blocks and not k_pool[0].is_contiguous():
+        raise ValueError("each pool block must be contiguous")
+    return num_blocks, block_size, k_pool.stride(0)
+
+
+def fp8_kv_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                 k_pool: torch.Tensor, v_pool: torch.Tensor, k_scale: float = 1.0,
+                 v_scale: float = 1.0, scale_dev: torch.Tensor | None = None, stream=None):
+    """reshape_and_cache_fp8: K, V ``[T, heads, dim]`` bf16 into the pools at
+    ``slot_mapping`` (int64, -1 skips), per-tensor scales by value or from the
+    device ``scale_dev [2]``."""
+    t, ks, e = _bf16_rows(k, "k")
+    t2, vs, e2 = _bf16_rows(v, "v")
+    if (t, e) != (t2, e2) or k.dim() != 3:
+        raise ValueError("k and v must both be [T, heads, dim]")
+    heads, dim = k.shape[1], k.shape[2]
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() < t:
+        raise ValueError("slot_mapping must be int64 with one entry per token")
+    nb, bs, cs = _pool_geometry(k_pool, v_pool, e)
+    _check("fp8_kv_write", lib.fp8_kv_write(
+        _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, heads, dim, _ptr(k_pool),
+        _ptr(v_pool), bs, cs, nb, float(k_scale), float(v_scale), _ptr(scale_dev),
+        _stream(stream)))
+
+
+def fp8_kv_amax_observe(k: torch.Tensor, v: torch.Tensor, amax_dev: torch.Tensor, stream=None):
+    """Max-accumulate max|K| and max|V| into the device fp32 ``amax_dev [2]``."""
+    t, ks, e = _bf16_rows(k, "k")
+    _, vs, _ = _bf16_rows(v, "v")
+    if amax_dev.dtype != torch.float32 or amax_dev.numel() < 2:
+        raise ValueError("amax_dev must be a float32 tensor of 2 elements")
+    _check("fp8_kv_amax_observe", lib.fp8_kv_amax_observe(
+        _ptr(k), _ptr(v), ks, vs, t, k.shape[1], k.shape[2], _ptr(amax_dev), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# calibration
+
+
+def fp8_kv_graphs_ready(states) -> bool:
+    """``states``: per layer None (no calibrator), False (in window), True (frozen)."""
+    arr = (ctypes.c_int8 * len(states))(*[-1 if s is None else int(bool(s)) for s in states])
+    r = lib.fp8_kv_graphs_ready(arr, len(states))
+    if r < 0:
+        raise Fp8qError("fp8_kv_graphs_ready", r, "invalid argument")
+    return bool(r)
+
+
+class KvCalibration:
+    """The calibrator of one attention layer (fp8_kv_calib_* of the C ABI).
+
+    Device memory (staging for the window's bf16 K/V and slots, and the
+    16-byte state) is allocated here with torch and handed to the library."""
+
+    def __init__(self, window_tokens: int, headroom: float, num_kv_heads: int, head_dim: int,
+                 device, stage_capacity: int | None = None, stream=None,
+                 state: torch.Tensor | None = None) -> None:
+        self.num_kv_heads = num_kv_heads
+        self.head_dim = head_dim
+        e = num_kv_heads * head_dim
+        window = min(int(window_tokens), MAX_STAGED_TOKENS)
+        cap = window if stage_capacity is None else int(stage_capacity)
+        self.stage_k = torch.empty((max(cap, 1), e), dtype=torch.bfloat16, device=device)
+        self.stage_v = torch.empty((max(cap, 1), e), dtype=torch.bfloat16, device=device)
+        self.stage_slots = torch.empty(max(cap, 1), dtype=torch.int64, device=device)
+        if state is None:
+            state = torch.empty(4, dtype=torch.float32, device=device)
+        if state.dtype != torch.float32 or state.numel() != 4 or not state.is_contiguous():
+            raise ValueError("state must be a contiguous float32 tensor of 4 elements")
+        self.state = state
+        self._h = ctypes.c_void_p()
+        self.handle = None
+        _check("fp8_kv_calib_create", lib.fp8_kv_calib_create(
+            int(window_tokens), float(headroom), num_kv_heads, head_dim, _ptr(self.stage_k),
+            _ptr(self.stage_v), _ptr(self.stage_slots), cap, _ptr(self.state), _stream(stream),
+            ctypes.byref(self._h)))
+        self.handle = self._h.value
+
+    def close(self) -> None:
+        if self.handle:
+            lib.fp8_kv_calib_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def scale_dev(self) -> torch.Tensor:
+        """Device ``{k_scale, v_scale}``: provisional until the freeze, frozen after."""
+        return self.state[2:4]
+
+    def observe(self, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                stream=None) -> int:
+        t, ks, e = _bf16_rows(k, "k")
+        _, vs, _ = _bf16_rows(v, "v")
+        step = ctypes.c_int32()
+        _check("fp8_kv_calib_observe", lib.fp8_kv_calib_observe(
+            self.handle, _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, k.shape[1],
+            k.shape[2], _stream(stream), ctypes.byref(step)))
+        return step.value
+
+    def freeze_replay(self, k_pool: torch.Tensor, v_pool: torch.Tensor, stream=None) -> int:
+        nb, bs, cs = _pool_geometry(k_pool, v_pool, self.num_kv_heads * self.head_dim)
+        n = ctypes.c_int64()
+        _check("fp8_kv_freeze_replay", lib.fp8_kv_freeze_replay(
+            self.handle, _ptr(k_pool), _ptr(v_pool), bs, cs, nb, _stream(stream),
+            ctypes.byref(n)))
+        return n.value
+
+    def observe_write(self, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                      k_pool: torch.Tensor, v_pool: torch.Tensor, stream=None) -> int:
+        t, ks, e = _bf16_rows(k, "k")
+        _, vs, _ = _bf16_rows(v, "v")
+        nb, bs, cs = _pool_geometry(k_pool, v_pool, e)
+        step = ctypes.c_int32()
+        _check("fp8_kv_calib_observe_write", lib.fp8_kv_calib_observe_write(
+            self.handle, _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, k.shape[1],
+            k.shape[2], _ptr(k_pool), _ptr(v_pool), bs, cs, nb, _stream(stream),
+            ctypes.byref(step)))
+        return step.value
+
+    def stats(self) -> dict:
+        s = CalibStats()
+        _check("fp8_kv_calib_stats_get", lib.fp8_kv_calib_stats_get(self.handle, ctypes.byref(s)))
+        return {name: getattr(s, name) for name, _ in CalibStats._fields_}
+
+    def read_state(self, stream=None):
+        """(k_amax, v_amax, k_scale, v_scale); synchronizes the stream."""
+        out = (ctypes.c_float * 4)()
+        _check("fp8_kv_calib_read_state", lib.fp8_kv_calib_read_state(
+            self.handle, _stream(stream), out))
+        return tuple(out)
+
+
+def fp8q_device_error(clear: bool = True) -> int:
+    """Sticky device error bits of the current device (synchronizes)."""
+    bits = ctypes.c_uint32()
+    _check("fp8q_device_error", lib.fp8q_device_error(ctypes.byref(bits), int(clear)))
+    return bits.value
+
+
+def version() -> int:
+    return lib.fp8q_version()
+
+
+def launch_count() -> int:
+    """Kernels the library has launched (or recorded into a graph) so far."""
+    return lib.fp8q_launch_count()
+
+
+# Module-level spellings of the calibrator entry points, with the C ABI's names.
+def fp8_kv_calib_create(window_tokens: int, headroom: float, num_kv_heads: int, head_dim: int,
+                        device, stage_capacity: int | None = None, stream=None) -> KvCalibration:
+    return KvCalibration(window_tokens, headroom, num_kv_heads, head_dim, device,
+                         stage_capacity, stream)
+
+
+def fp8_kv_calib_observe(calib: KvCalibration, k, v, slot_mapping, stream=None) -> int:
+    return calib.observe(k, v, slot_mapping, stream)
+
+
+def fp8_kv_freeze_replay(calib: KvCalibration, k_pool, v_pool, stream=None) -> int:
+    return calib.freeze_replay(k_pool, v_pool, stream)
+
+
+def fp8_kv_calib_observe_write(calib: KvCalibration, k, v, slot_mapping, k_pool, v_pool,
+                               stream=None) -> int:
+    return calib.observe_write(k, v, slot_mapping, k_pool, v_pool, stream)

@@ -1,0 +1,74 @@
+// Internal interface between the C ABI (fp8q_api.cpp) and the kernels
+// (fp8q_kernels.cu).  Not installed; the public surface is include/fp8q.h.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace fp8q {
+
+// One pass of the KV kernel over a batch of tokens.  Which of the three jobs
+// it does is chosen by the flags; every job reads each K/V row once.
+//   amax   max-accumulate |K|, |V| (fp32 bit patterns) into amax_bits[0..1]
+//   stage  copy the rows, packed, to stage_k/stage_v at row stage_offset + t,
+//          and the slot to stage_slots[stage_offset + t]
+//   write  quantize the rows and scatter them into the pools
+struct KvPass {
+    const uint16_t *k = nullptr;
+    const uint16_t *v = nullptr;
+    int64_t key_stride = 0;
+    int64_t value_stride = 0;
+    const int64_t *slot_mapping = nullptr;
+    int64_t num_tokens = 0;
+    int32_t elems = 0;  // num_kv_heads * head_dim, a multiple of 8
+
+    // write
+    uint8_t *k_pool = nullptr;
+    uint8_t *v_pool = nullptr;
+    int32_t block_size = 0;
+    int64_t cache_stride = 0;
+    int64_t num_slots = 0;
+    // Scale source, first match wins:
+    //   freeze_amax != null: scale = max(amax*headroom, 1e-12)/448 from the
+    //                        accumulated maxima; block 0 stores it to scale_out
+    //   scale_dev   != null: {k_scale, v_scale} read from device memory
+    //   otherwise           k_scale / v_scale by value
+    const uint32_t *freeze_amax = nullptr;
+    float headroom = 1.0f;
+    float *scale_out = nullptr;
+    const float *scale_dev = nullptr;
+    float k_scale = 1.0f;
+    float v_scale = 1.0f;
+
+    // amax
+    uint32_t *amax_bits = nullptr;
+
+    // stage
+    uint16_t *stage_k = nullptr;
+    uint16_t *stage_v = nullptr;
+    int64_t *stage_slots = nullptr;
+    int64_t stage_offset = 0;
+
+    bool do_amax = false;
+    bool do_stage = false;
+    bool do_write = false;
+};
+
+cudaError_t launch_group_quant(const uint16_t *x, int64_t x_row_stride, uint8_t *q,
+                               float *scales, int64_t m, int64_t k, cudaStream_t stream);
+
+// Launches one KV pass.  A pass with no tokens still launches when it must
+// publish a frozen scale (freeze_amax and scale_out set).
+cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream);
+
+// Enqueues state_dev = {0, 0, 2.0, 2.0} (bit patterns of the fp32 values).
+cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream);
+
+// Number of kernels this library has launched in this process.
+int64_t launch_count();
+
+// Sticky device error word of the current device.
+cudaError_t read_device_error(uint32_t *bits, bool clear);
+
+}  // namespace fp8q

@@ -1,0 +1,509 @@
+// fp8q_kernels.cu -- sm_100a kernels of the FP8 E4M3 quantization path.
+//
+// All three kernels are bound by HBM bandwidth: every element is read once
+// (bf16, 2 B) and written once (E4M3, 1 B) with a handful of ALU operations in
+// between.  Nothing here is a contraction, so there are no tensor-core paths;
+// the design goals are fully coalesced 128-bit loads, enough bytes in flight
+// per SM to cover HBM latency, and an encode that is exact yet cheap.
+//
+// Exact arithmetic.  A code is E4M3(fp32(x / s)).  The fp32 quotient is
+// formed from r = RN(1/s) (one IEEE reciprocal per group or per tensor) with
+// one product and one FMA correction:
+//     q0 = RN(x * r);  e = x - q0*s (exact in an FMA);  q = RN(q0 + e*r)
+// By Markstein's theorem (r within half an ulp of 1/s, q0 within one ulp of
+// x/s, no underflow or overflow) q is the correctly rounded x/s.  The
+// magnitude is then given the sign of x, so -0 stays -0.  For the activation
+// quantizer this was checked exhaustively over every pair of bf16 x and bf16
+// group maximum; for a per-tensor scale the fast form is used only while the
+// scale lies in [2^-64, 2^64] (x clamped so that x * r cannot overflow, which
+// only changes values that saturate anyway), and __fdiv_rn is used outside
+// that range.  The quotient is then rounded by the hardware conversion
+// cvt.rn.satfinite.e4m3x2.f32: nearest-even, saturating to +-448.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "fp8q_internal.h"
+
+namespace fp8q {
+
+// Kernels launched by this library in this process (diagnostics).
+std::atomic<int64_t> g_launch_count{0};
+
+// Sticky error word of this device (one per device that loads the library).
+__device__ uint32_t g_error_word;
+
+namespace {
+
+constexpr float kE4m3Max = 448.0f;
+constexpr float kScaleFloor = 1e-12f;
+constexpr uint32_t kErrSlot = 0x1u;
+constexpr uint32_t kErrScale = 0x2u;
+
+// ---------------------------------------------------------------------------
+// device helpers
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 128-bit load of data read exactly once: no L1 allocation.  volatile: the
+// load must never be hoisted above the bounds test that guards it.
+__device__ __forceinline__ uint4 ld_once(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+// Per-half max of |a| and |b| for two bf16x2 words (the sign bits of the
+// result carry no meaning and are cleared by the caller).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t absmax_uint4(uint32_t acc, const uint4 &c) {
+    acc = absmax_bf16x2(acc, c.x);
+    acc = absmax_bf16x2(acc, c.y);
+    acc = absmax_bf16x2(acc, c.z);
+    acc = absmax_bf16x2(acc, c.w);
+    return acc;
+}
+
+// Largest |value| of a bf16x2 accumulator, as the 16-bit magnitude pattern.
+__device__ __forceinline__ uint32_t absmax_bits16(uint32_t acc) {
+    acc &= 0x7FFF7FFFu;
+    return max(acc & 0xFFFFu, acc >> 16);
+}
+
+__device__ __forceinline__ uint32_t clamp_bf16x2(uint32_t w, uint32_t lo2, uint32_t hi2) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(w), "r"(lo2));
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(d), "r"(hi2));
+    return d;
+}
+
+// Two fp32 values to two E4M3 codes: byte 0 <- lo, byte 1 <- hi.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    unsigned short d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+struct Divisor {
+    float s;     // the scale
+    float r;     // RN(1/s)
+};
+
+// Correctly rounded x / s (see the file comment), sign of x.
+__device__ __forceinline__ float quotient(float x, const Divisor &d) {
+    const float q0 = __fmul_rn(x, d.r);
+    const float e = __fmaf_rn(-q0, d.s, x);
+    const float q = __fmaf_rn(e, d.r, q0);
+    return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) |
+                           (__float_as_uint(x) & 0x80000000u));
+}
+
+__device__ __forceinline__ uint2 encode8(const uint4 &w, const Divisor &d) {
+    uint2 o;
+    o.x = e4m3x2(quotient(bf16_lo(w.x), d), quotient(bf16_hi(w.x), d)) |
+          (e4m3x2(quotient(bf16_lo(w.y), d), quotient(bf16_hi(w.y), d)) << 16);
+    o.y = e4m3x2(quotient(bf16_lo(w.z), d), quotient(bf16_hi(w.z), d)) |
+          (e4m3x2(quotient(bf16_lo(w.w), d), quotient(bf16_hi(w.w), d)) << 16);
+    return o;
+}
+
+// IEEE division per element, for scales outside the fast range.
+__device__ __forceinline__ uint2 encode8_div(const uint4 &w, float s) {
+    uint2 o;
+    o.x = e4m3x2(__fdiv_rn(bf16_lo(w.x), s), __fdiv_rn(bf16_hi(w.x), s)) |
+          (e4m3x2(__fdiv_rn(bf16_lo(w.y), s), __fdiv_rn(bf16_hi(w.y), s)) << 16);
+    o.y = e4m3x2(__fdiv_rn(bf16_lo(w.z), s), __fdiv_rn(bf16_hi(w.z), s)) |
+          (e4m3x2(__fdiv_rn(bf16_lo(w.w), s), __fdiv_rn(bf16_hi(w.w), s)) << 16);
+    return o;
+}
+
+// Per-tensor encoder: fast path with a clamp, or IEEE division.
+struct TensorEncoder {
+    Divisor d;
+    uint32_t lo2, hi2;   // clamp bounds as bf16x2 (-T, T)
+    bool fast;
+    bool ok;             // scale is a positive number
+
+    __device__ __forceinline__ void init(float s) {
+        ok = s > 0.0f;   // false for NaN
+        fast = (s >= 0x1p-64f) && (s <= 0x1p64f);
+        d.s = s;
+        d.r = __frcp_rn(s);
+        // T = s * 1024 rounded up to bf16: any |x| >= T saturates, and T * r
+        // stays far from overflow.
+        uint32_t u = __float_as_uint(__fmul_rn(s, 1024.0f));
+        if (u & 0xFFFFu) u += 0x10000u;
+        const uint32_t t = (u >> 16) & 0x7FFFu;
+        hi2 = t | (t << 16);
+        lo2 = hi2 | 0x80008000u;
+    }
+
+    __device__ __forceinline__ uint2 encode(uint4 w) const {
+        if (fast) {
+            w.x = clamp_bf16x2(w.x, lo2, hi2);
+            w.y = clamp_bf16x2(w.y, lo2, hi2);
+            w.z = clamp_bf16x2(w.z, lo2, hi2);
+            w.w = clamp_bf16x2(w.w, lo2, hi2);
+            return encode8(w, d);
+        }
+        return encode8_div(w, d.s);
+    }
+};
+
+// Frozen scale: max(amax * headroom, 1e-12) / 448, product rounded first.
+__device__ __forceinline__ float freeze_scale(uint32_t amax_bits, float headroom) {
+    const float widened = __fmul_rn(__uint_as_float(amax_bits), headroom);
+    return __fdiv_rn(fmaxf(widened, kScaleFloor), kE4m3Max);
+}
+
+// ---------------------------------------------------------------------------
+// 1. per-token 1x128-group quantization
+//
+// Four lanes own one 128-element group (32 elements each); a warp covers
+// eight consecutive groups (2 KB of input).  Lane q of a group loads chunks
+// q, q+4, q+8, q+12 of 16 bytes, so each of the four load instructions of a
+// warp reads eight fully used 64-byte runs, and each store writes eight full
+// 32-byte sectors.  The group maximum needs two shuffles.
+
+constexpr int kGqThreads = 256;
+
+template <bool kPacked>
+__global__ void __launch_bounds__(kGqThreads)
+group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
+                   uint8_t *__restrict__ q, float *__restrict__ scales,
+                   int64_t total_groups, uint32_t groups_per_row) {
+    const int lane = threadIdx.x & 31;
+    const int sub = lane >> 2;   // group within the warp's eight
+    const int ql = lane & 3;     // lane within the group
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kGqThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGqThreads) >> 5;
+    const int64_t octets = (total_groups + 7) >> 3;
+
+    for (int64_t o = warp; o < octets; o += nwarps) {
+        const int64_t g = o * 8 + sub;
+        const bool valid = g < total_groups;
+        const uint16_t *src;
+        if (kPacked) {
+            src = x + g * 128;
+        } else {
+            const uint64_t row = static_cast<uint64_t>(g) / groups_per_row;
+            src = x + row * x_row_stride + (static_cast<uint64_t>(g) - row * groups_per_row) * 128;
+        }
+        uint4 c[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            c[j] = valid ? ld_once(src + (ql + 4 * j) * 8) : make_uint4(0, 0, 0, 0);
+
+        uint32_t acc = c[0].x;
+        acc = absmax_bf16x2(acc, c[0].y);
+        acc = absmax_bf16x2(acc, c[0].z);
+        acc = absmax_bf16x2(acc, c[0].w);
+#pragma unroll
+        for (int j = 1; j < 4; ++j) acc = absmax_uint4(acc, c[j]);
+        uint32_t m = absmax_bits16(acc);
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+
+        const float amax = __uint_as_float(m << 16);
+        Divisor d;
+        d.s = __fdiv_rn(fmaxf(amax, kScaleFloor), kE4m3Max);
+        d.r = __frcp_rn(d.s);
+
+        if (valid) {
+            uint8_t *dst = q + g * 128;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) = encode8(c[j], d);
+            if (ql == 0) scales[g] = d.s;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2./3. KV pass: absmax, staging copy and quantize-and-scatter
+//
+// One warp per token (grid-stride).  Lane l owns 16-byte chunks l and l+32 of
+// the K row and of the V row, so every load and store instruction of the warp
+// is one contiguous run (512 B of bf16 in, 256 B of codes out).  The slot
+// decides where the codes land: one token's entry is E contiguous bytes of the
+// pool, written as 32 8-byte stores per instruction.
+
+constexpr int kKvThreads = 256;
+constexpr int kKvWarps = kKvThreads / 32;
+
+template <bool kAmax, bool kStage, bool kWrite>
+__global__ void __launch_bounds__(kKvThreads) kv_pass_kernel(const KvPass p) {
+    TensorEncoder kenc, venc;
+    if (kWrite) {
+        float ks, vs;
+        if (p.freeze_amax != nullptr) {
+            ks = freeze_scale(p.freeze_amax[0], p.headroom);
+            vs = freeze_scale(p.freeze_amax[1], p.headroom);
+            if (p.scale_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+                p.scale_out[0] = ks;
+                p.scale_out[1] = vs;
+            }
+        } else if (p.scale_dev != nullptr) {
+            ks = p.scale_dev[0];
+            vs = p.scale_dev[1];
+        } else {
+            ks = p.k_scale;
+            vs = p.v_scale;
+        }
+        kenc.init(ks);
+        venc.init(vs);
+        if (!(kenc.ok && venc.ok) && blockIdx.x == 0 && threadIdx.x == 0)
+            atomicOr(&g_error_word, kErrScale);
+    }
+
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kKvThreads) >> 5;
+    const int nchunks = p.elems >> 3;
+    const bool small_slots = p.num_slots <= 0x7FFFFFFF;
+    uint32_t kacc = 0, vacc = 0;
+
+    for (int64_t t = warp; t < p.num_tokens; t += nwarps) {
+        int64_t slot = -1;
+        if (kWrite || kStage) slot = __ldg(p.slot_mapping + t);
+        bool write_row = false;
+        int64_t dst = 0;
+        if (kWrite && slot >= 0) {
+            if (slot >= p.num_slots) {
+                if (lane == 0) atomicOr(&g_error_word, kErrSlot);
+            } else {
+                int64_t blk, off;
+                if (small_slots) {
+                    const uint32_t s32 = static_cast<uint32_t>(slot);
+                    const uint32_t b32 = s32 / static_cast<uint32_t>(p.block_size);
+                    blk = b32;
+                    off = s32 - b32 * static_cast<uint32_t>(p.block_size);
+                } else {
+                    blk = slot / p.block_size;
+                    off = slot - blk * p.block_size;
+                }
+                dst = blk * p.cache_stride + off * p.elems;
+                write_row = true;
+            }
+        }
+        const uint16_t *krow = p.k + t * p.key_stride;
+        const uint16_t *vrow = p.v + t * p.value_stride;
+
+        for (int c0 = 0; c0 < nchunks; c0 += 64) {
+            const int ca = c0 + lane;
+            const int cb = c0 + 32 + lane;
+            const bool ha = ca < nchunks;
+            const bool hb = cb < nchunks;
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            const uint4 ka = ha ? ld_once(krow + ca * 8) : z;
+            const uint4 kb = hb ? ld_once(krow + cb * 8) : z;
+            const uint4 va = ha ? ld_once(vrow + ca * 8) : z;
+            const uint4 vb = hb ? ld_once(vrow + cb * 8) : z;
+            if (kAmax) {
+                kacc = absmax_uint4(absmax_uint4(kacc, ka), kb);
+                vacc = absmax_uint4(absmax_uint4(vacc, va), vb);
+            }
+            if (kStage) {
+                const int64_t row = (p.stage_offset + t) * p.elems;
+                if (ha) {
+                    *reinterpret_cast<uint4 *>(p.stage_k + row + ca * 8) = ka;
+                    *reinterpret_cast<uint4 *>(p.stage_v + row + ca * 8) = va;
+                }
+                if (hb) {
+                    *reinterpret_cast<uint4 *>(p.stage_k + row + cb * 8) = kb;
+                    *reinterpret_cast<uint4 *>(p.stage_v + row + cb * 8) = vb;
+                }
+            }
+            if (kWrite && write_row) {
+                if (kenc.ok) {
+                    if (ha) *reinterpret_cast<uint2 *>(p.k_pool + dst + ca * 8) = kenc.encode(ka);
+                    if (hb) *reinterpret_cast<uint2 *>(p.k_pool + dst + cb * 8) = kenc.encode(kb);
+                }
+                if (venc.ok) {
+                    if (ha) *reinterpret_cast<uint2 *>(p.v_pool + dst + ca * 8) = venc.encode(va);
+                    if (hb) *reinterpret_cast<uint2 *>(p.v_pool + dst + cb * 8) = venc.encode(vb);
+                }
+            }
+        }
+        if (kStage && lane == 0) p.stage_slots[p.stage_offset + t] = slot;
+    }
+
+    if (kAmax) {
+        __shared__ uint32_t red[2][kKvWarps];
+        uint32_t km = __reduce_max_sync(0xFFFFFFFFu, absmax_bits16(kacc));
+        uint32_t vm = __reduce_max_sync(0xFFFFFFFFu, absmax_bits16(vacc));
+        const int w = threadIdx.x >> 5;
+        if (lane == 0) {
+            red[0][w] = km;
+            red[1][w] = vm;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+#pragma unroll
+            for (int i = 1; i < kKvWarps; ++i) {
+                km = max(km, red[0][i]);
+                vm = max(vm, red[1][i]);
+            }
+            // fp32 bit patterns of non-negative values order like unsigned
+            // integers, so an integer atomicMax is a float max here.
+            if (km) atomicMax(p.amax_bits + 0, km << 16);
+            if (vm) atomicMax(p.amax_bits + 1, vm << 16);
+        }
+    }
+}
+
+__global__ void calib_init_kernel(float *state) {
+    state[0] = 0.0f;
+    state[1] = 0.0f;
+    state[2] = 2.0f;
+    state[3] = 2.0f;
+}
+
+// ---------------------------------------------------------------------------
+// launch geometry
+
+struct DeviceInfo {
+    int sms = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_info_mutex;
+DeviceInfo g_info[kMaxDevices];
+
+cudaError_t device_sms(int *sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_info_mutex);
+    if (g_info[dev].sms == 0) {
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        g_info[dev].sms = n;
+    }
+    *sms = g_info[dev].sms;
+    return cudaSuccess;
+}
+
+// Resident CTAs per SM of a kernel, cached per (device, kernel).
+std::mutex g_occ_mutex;
+std::map<std::pair<int, const void *>, int> g_occ;
+
+template <typename Kernel>
+cudaError_t resident_ctas(Kernel kernel, int threads, int *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kernel));
+    std::lock_guard<std::mutex> lock(g_occ_mutex);
+    auto it = g_occ.find(key);
+    if (it == g_occ.end()) {
+        int n = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0);
+        if (e != cudaSuccess) return e;
+        it = g_occ.emplace(key, n > 0 ? n : 1).first;
+    }
+    *out = it->second;
+    return cudaSuccess;
+}
+
+template <typename Kernel>
+cudaError_t grid_for(Kernel kernel, int threads, int64_t ctas_wanted, int *grid) {
+    int sms = 0, per_sm = 0;
+    cudaError_t e = device_sms(&sms);
+    if (e != cudaSuccess) return e;
+    e = resident_ctas(kernel, threads, &per_sm);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+    int64_t g = ctas_wanted < cap ? ctas_wanted : cap;
+    if (g < 1) g = 1;
+    *grid = static_cast<int>(g);
+    return cudaSuccess;
+}
+
+template <bool A, bool S, bool W>
+cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
+    auto kernel = kv_pass_kernel<A, S, W>;
+    const int64_t wanted = (p.num_tokens + kKvWarps - 1) / kKvWarps;
+    int grid = 1;
+    cudaError_t e = grid_for(kernel, kKvThreads, wanted, &grid);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kKvThreads, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) g_launch_count.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
+}  // namespace
+
+cudaError_t launch_group_quant(const uint16_t *x, int64_t x_row_stride, uint8_t *q,
+                               float *scales, int64_t m, int64_t k, cudaStream_t stream) {
+    const int64_t gpr = k / 128;
+    const int64_t total = m * gpr;
+    if (total == 0) return cudaSuccess;
+    const int64_t warps = (total + 7) / 8;
+    const int64_t wanted = (warps * 32 + kGqThreads - 1) / kGqThreads;
+    int grid = 1;
+    cudaError_t e;
+    if (x_row_stride == k) {
+        e = grid_for(group_quant_kernel<true>, kGqThreads, wanted, &grid);
+        if (e != cudaSuccess) return e;
+        group_quant_kernel<true><<<grid, kGqThreads, 0, stream>>>(
+            x, x_row_stride, q, scales, total, static_cast<uint32_t>(gpr));
+    } else {
+        e = grid_for(group_quant_kernel<false>, kGqThreads, wanted, &grid);
+        if (e != cudaSuccess) return e;
+        group_quant_kernel<false><<<grid, kGqThreads, 0, stream>>>(
+            x, x_row_stride, q, scales, total, static_cast<uint32_t>(gpr));
+    }
+    e = cudaGetLastError();
+    if (e == cudaSuccess) g_launch_count.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
+cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
+    const bool publish = p.do_write && p.freeze_amax != nullptr && p.scale_out != nullptr;
+    if (p.num_tokens == 0 && !publish) return cudaSuccess;
+    if (p.do_amax && p.do_stage && p.do_write) return launch_kv_variant<true, true, true>(p, stream);
+    if (p.do_amax && p.do_stage) return launch_kv_variant<true, true, false>(p, stream);
+    if (p.do_amax && p.do_write) return launch_kv_variant<true, false, true>(p, stream);
+    if (p.do_amax) return launch_kv_variant<true, false, false>(p, stream);
+    if (p.do_write) return launch_kv_variant<false, false, true>(p, stream);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream) {
+    calib_init_kernel<<<1, 1, 0, stream>>>(state_dev);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) g_launch_count.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
+int64_t launch_count() { return g_launch_count.load(std::memory_order_relaxed); }
+
+cudaError_t read_device_error(uint32_t *bits, bool clear) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(bits, g_error_word, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    if (clear) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(uint32_t));
+    }
+    return e;
+}
+
+}  // namespace fp8q

@@ -1,0 +1,212 @@
+"""GPU parity of the calibration window (observe, staging, freeze, replay,
+crossing write) against the oracle's restatement of the pages' algorithm:
+the pools after every batch, the steps, the frozen scales and the counters
+must all agree exactly."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_group_b200 as fp8q
+import workloads
+from gpu_util import dev, dev_bf16, first_mismatch, host
+from oracle import calibration as cal
+
+pytestmark = pytest.mark.gpu
+
+STEP_NAMES = {fp8q.STEP_STAGE: cal.STAGE, fp8q.STEP_STAGE_DECLINED: cal.STAGE,
+              fp8q.STEP_FREEZE: cal.FREEZE, fp8q.STEP_FROZEN: cal.FROZEN}
+
+
+def _rows(bits, heads, dim):
+    t, stride = bits.shape
+    return dev_bf16(bits).as_strided((t, heads, dim), (stride, dim, 1))
+
+
+class GpuLayer:
+    """One layer's pools on the device and the calibrator, driven the way the
+    attention write path drives it."""
+
+    def __init__(self, spec, window, headroom, fused, stage_capacity=None):
+        self.spec = spec
+        self.fused = fused
+        n = spec.num_blocks * spec.cache_stride
+        self.kp = torch.full((n,), workloads.SENTINEL, dtype=torch.uint8, device="cuda")
+        self.vp = torch.full((n,), workloads.SENTINEL, dtype=torch.uint8, device="cuda")
+        shape = (spec.num_blocks, spec.block_size, spec.heads, spec.dim)
+        self.kp4, self.vp4 = self.kp.view(shape), self.vp.view(shape)
+        self.cal = fp8q.KvCalibration(window, headroom, spec.heads, spec.dim, "cuda",
+                                      stage_capacity=stage_capacity)
+
+    def step(self, b):
+        k, v = _rows(b.k, self.spec.heads, self.spec.dim), _rows(b.v, self.spec.heads, self.spec.dim)
+        slots = dev(b.slot_mapping)
+        if self.fused:
+            return self.cal.observe_write(k, v, slots, self.kp4, self.vp4)
+        step = self.cal.observe(k, v, slots)
+        if step == fp8q.STEP_FREEZE:
+            self.cal.freeze_replay(self.kp4, self.vp4)
+        fp8q.fp8_kv_write(k, v, slots, self.kp4, self.vp4, scale_dev=self.cal.scale_dev)
+        return step
+
+
+def _oracle_layer(spec, window, headroom, stage_capacity=None):
+    c = cal.Fp8KvCalibration(0, window, headroom, staging_capacity=stage_capacity)
+    kp, vp = spec.new_pool().reshape(-1), spec.new_pool().reshape(-1)
+    return c, kp, vp
+
+
+def _run_both(spec, batches, window, headroom, fused, stage_capacity=None, check_every=True):
+    g = GpuLayer(spec, window, headroom, fused, stage_capacity)
+    c, kp, vp = _oracle_layer(spec, window, headroom, stage_capacity)
+    steps = []
+    for i, b in enumerate(batches):
+        gs = g.step(b)
+        run = cal.run_calibrated_writes(
+            c, [cal.KvBatch(b.k, b.v, b.slot_mapping, b.key_stride, b.value_stride)],
+            spec.heads, spec.dim, kp, vp, spec.block_size, spec.cache_stride, spec.num_blocks)
+        assert STEP_NAMES[gs] == run.steps[0], (i, gs, run.steps[0])
+        steps.append(gs)
+        if check_every or i == len(batches) - 1:
+            gk, gv = host(g.kp), host(g.vp)
+            assert np.array_equal(gk, kp), f"batch {i}: " + first_mismatch(gk, kp)
+            assert np.array_equal(gv, vp), f"batch {i}: " + first_mismatch(gv, vp)
+    return g, c, steps
+
+
+def _assert_frozen_state(g, c):
+    ka, va, ks, vs = g.cal.read_state()
+    assert np.float32(ka) == c.state.k_running_max and np.float32(va) == c.state.v_running_max
+    assert (np.float32(ks), np.float32(vs)) == c.scales()
+    st = g.cal.stats()
+    log = c.freeze_log
+    assert st["state"] == 2
+    assert st["freeze_tokens"] == log.tokens_seen
+    assert st["replayed_tokens"] == log.staged_tokens
+    assert st["staged_batches"] == log.staged_batches
+    assert st["unstaged_tokens"] == log.unstaged_tokens
+    assert st["window_tokens"] == c.state.window_tokens
+    assert st["requested_tokens"] == c.requested_tokens
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_calibration_window_workload(fused):
+    spec, batches, _ = workloads.calib_window()
+    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused)
+    assert steps == [fp8q.STEP_STAGE] * 8 + [fp8q.STEP_FREEZE] + [fp8q.STEP_FROZEN] * 2
+    _assert_frozen_state(g, c)
+    assert g.cal.read_state()[2] == np.float32(np.float32(600.0) / np.float32(448.0))
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_strided_sources_and_headroom(fused):
+    spec, batches, _ = workloads.calib_window(row_pad=40)
+    g, c, _ = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.25, fused)
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_declined_batches(fused):
+    spec, batches, _ = workloads.calib_window()
+    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused, stage_capacity=60)
+    assert steps[:8] == [fp8q.STEP_STAGE] * 2 + [fp8q.STEP_STAGE_DECLINED] * 6
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_window_of_one_and_exact_window(fused):
+    spec, batches, _ = workloads.calib_window(batch_sizes=(13, 32, 32))
+    g, c, steps = _run_both(spec, batches, 1, 0.5, fused)
+    assert steps == [fp8q.STEP_FREEZE, fp8q.STEP_FROZEN, fp8q.STEP_FROZEN]
+    _assert_frozen_state(g, c)
+    g, c, steps = _run_both(spec, batches, 45, 1.0, fused)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_FREEZE, fp8q.STEP_FROZEN]
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("layer", [0, 7])
+def test_large_prefill_chunked_replay(fused, layer):
+    """4095 staged tokens (the cap), then the 498-token crossing chunk."""
+    spec = workloads.large_kv_spec()
+    full = workloads.large_kv_layer(layer)
+    chunks = workloads.split_batch(full, workloads.LARGE_CHUNKS)
+    g, c, steps = _run_both(spec, chunks, workloads.LARGE_WINDOW_REQUEST, 1.0, fused,
+                            check_every=False)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
+    _assert_frozen_state(g, c)
+    assert g.cal.stats()["replayed_tokens"] == 4095
+    assert g.cal.stats()["window_tokens"] == 4096
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_large_prefill_single_chunk_freezes_at_once(fused):
+    spec = workloads.large_kv_spec()
+    full = workloads.large_kv_layer(3)
+    g, c, steps = _run_both(spec, [full], workloads.LARGE_WINDOW_REQUEST, 1.0, fused)
+    assert steps == [fp8q.STEP_FREEZE]
+    assert g.cal.stats()["replayed_tokens"] == 0
+    _assert_frozen_state(g, c)
+
+
+def test_zero_token_observe_counts_a_stage_step():
+    spec, batches, _ = workloads.calib_window(batch_sizes=(13, 32))
+    empty = workloads.KvBatchInput(batches[0].k[:0], batches[0].v[:0],
+                                   batches[0].slot_mapping[:0], 512, 512)
+    g, c, steps = _run_both(spec, [batches[0], empty, batches[1]], 40, 1.0, fused=False)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
+    _assert_frozen_state(g, c)
+
+
+def test_calls_out_of_order_are_rejected():
+    spec, batches, _ = workloads.calib_window(batch_sizes=(13, 32, 32))
+    g = GpuLayer(spec, 40, 1.0, fused=False)
+    b0, b1 = batches[0], batches[1]
+    with pytest.raises(fp8q.Fp8qError) as ei:
+        g.cal.freeze_replay(g.kp4, g.vp4)          # nothing pending
+    assert ei.value.status == -3
+    k, v = _rows(b0.k, 4, 128), _rows(b0.v, 4, 128)
+    assert g.cal.observe(k, v, dev(b0.slot_mapping)) == fp8q.STEP_STAGE
+    k, v = _rows(b1.k, 4, 128), _rows(b1.v, 4, 128)
+    assert g.cal.observe(k, v, dev(b1.slot_mapping)) == fp8q.STEP_FREEZE
+    with pytest.raises(fp8q.Fp8qError) as ei:
+        g.cal.observe(k, v, dev(b1.slot_mapping))   # replay still pending
+    assert ei.value.status == -3
+    assert g.cal.freeze_replay(g.kp4, g.vp4) == 13
+    assert g.cal.observe(k, v, dev(b1.slot_mapping)) == fp8q.STEP_FROZEN
+
+
+def test_post_freeze_write_in_a_cuda_graph():
+    """After the freeze the write reads its scales from the device, so a graph
+    captured once keeps writing at whatever the calibrator published."""
+    spec, batches, _ = workloads.calib_window()
+    g = GpuLayer(spec, workloads.CALIB_WINDOW, 1.0, fused=False)
+    for b in batches[:9]:
+        g.step(b)
+    b = batches[9]
+    k, v = _rows(b.k, 4, 128), _rows(b.v, 4, 128)
+    slots = dev(b.slot_mapping)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        fp8q.fp8_kv_write(k, v, slots, g.kp4, g.vp4, scale_dev=g.cal.scale_dev, stream=s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=s):
+            fp8q.fp8_kv_write(k, v, slots, g.kp4, g.vp4, scale_dev=g.cal.scale_dev, stream=s)
+    eager = host(g.kp).copy()
+    # replay the graph into pools reset to the sentinel: exactly batch 10's
+    # entries come back, equal to the eager write
+    g.kp.fill_(workloads.SENTINEL)
+    g.vp.fill_(workloads.SENTINEL)
+    graph.replay()
+    torch.cuda.synchronize()
+    got = host(g.kp)
+    mask = np.zeros(got.size, bool)
+    for slot in b.slot_mapping:
+        blk, off = divmod(int(slot), spec.block_size)
+        base = blk * spec.cache_stride + off * spec.elems
+        mask[base:base + spec.elems] = True
+    assert np.array_equal(got[mask], eager[mask])
+    assert np.all(got[~mask] == workloads.SENTINEL)
+    del graph
