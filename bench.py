@@ -10,12 +10,14 @@ One step is one 4593-token prefill through every operation of the path:
     window (absmax; freeze and replay of the 4095 staged tokens; write of the
     crossing chunk at the frozen scale).
 That is 1 + 16 x 4 = 65 kernel launches, issued through the C ABI and
-replayed as one CUDA graph.  Before every step L2 is flushed (a 2x-L2 write)
-and the calibrators' device state is reset, both outside the timed region.
+replayed as one CUDA graph.  Before every step L2 is flushed (a 2x-L2 write,
+then a 2x-L2 read of a clean buffer) and the calibrators' device state is
+reset, both outside the timed region.
 
 `value` is effective HBM GB/s: the algorithmic bytes of the step (each
 kernel's compulsory reads and writes) divided by the step time measured with
-CUDA events.  Per-kernel times come from event nodes between the launches.
+CUDA events.  Per-kernel times come from graphs of each kernel's launches as
+the step issues them (one per layer, back to back), timed the same way.
 `--impl reference` times the CPU oracle on a bounded sample of the same step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
@@ -208,6 +210,7 @@ class Workload:
         self.states_init = torch.tensor([0.0, 0.0, 2.0, 2.0], device=device).repeat(layers, 1)
         l2 = torch.cuda.get_device_properties(device).L2_cache_size
         self.flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+        self.flush_read = torch.ones(2 * l2, dtype=torch.uint8, device=device)
 
     def _bf16(self, bits):
         t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
@@ -219,9 +222,16 @@ class Workload:
                                    workloads.HEAD_DIM, self.device, state=self.states[l])
                 for l in range(self.layers)]
 
+    def flush(self, i: int) -> None:
+        """Write 2x L2, then read another 2x L2 that is never written: L2 ends
+        up holding only clean lines of a buffer no kernel uses, so the timed
+        kernels neither hit in L2 nor pay for write-backs of dirty lines."""
+        self.flush_buf.fill_(i & 0xFF)
+        self._sink = torch.amax(self.flush_read)
+
     def reset(self, i: int) -> None:
         self.states.copy_(self.states_init)
-        self.flush_buf.fill_(i & 0xFF)
+        self.flush(i)
 
     def issue(self, calibs, mark) -> None:
         fp8q = self.fp8q
@@ -247,31 +257,93 @@ def labels_of(layers: int) -> list[str]:
     return ["group_quant"] + ["observe_stage_write", "amax", "freeze_replay", "kv_write"] * layers
 
 
-def capture(w: Workload, stream, with_events: bool):
-    """Capture one step into a CUDA graph; event nodes between launches."""
+def capture(w: Workload, stream):
+    """Capture one step into a CUDA graph (no event nodes: they would break
+    the programmatic overlap of consecutive launches)."""
     labels = labels_of(w.layers)
-    events = [torch.cuda.Event(enable_timing=True, external=True)
-              for _ in range(len(labels) + 1)] if with_events else []
     with torch.cuda.stream(stream):
         calibs = w.calibrators()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     before = w.fp8q.launch_count()
-    pos = [0]
-
-    def mark(_label):
-        if with_events:
-            pos[0] += 1
-            events[pos[0]].record()
-
     with torch.cuda.graph(graph, stream=stream):
-        if with_events:
-            events[0].record()
-        w.issue(calibs, mark)
+        w.issue(calibs, lambda _l: None)
     launches = w.fp8q.launch_count() - before
     # The graph writes into these calibrators' staging tensors on every
     # replay: the caller keeps them alive as long as the graph.
-    return graph, events, labels, launches, calibs
+    return graph, labels, launches, calibs
+
+
+def time_graph(w: Workload, stream, graph, reps: int, reset_state: bool) -> list[float]:
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            if reset_state:
+                w.reset(i)
+            else:
+                w.flush(i)
+            start.record()
+            graph.replay()
+            end.record()
+            end.synchronize()
+            out.append(start.elapsed_time(end))
+    return out
+
+
+def kernel_sequences(w: Workload, stream, reps: int) -> dict:
+    """Average launch duration of each kernel of the step, from a graph of its
+    launches exactly as the step issues them (one per layer, back to back),
+    the state before them prepared eagerly.  Returns {label: (us, launches)}."""
+    fp8q = w.fp8q
+    L = w.layers
+    out = {}
+
+    def chunks(l):
+        return (w.k[l], w.v[l], w.slots[l], w.k_pool[l], w.v_pool[l])
+
+    def stage_all(calibs):
+        for l, c in enumerate(calibs):
+            k, v, s, kp, vp = chunks(l)
+            c.observe_write(k[:CHUNK1], v[:CHUNK1], s[:CHUNK1], kp, vp)
+
+    def observe_all(calibs):
+        for l, c in enumerate(calibs):
+            k, v, s, _, _ = chunks(l)
+            c.observe(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:])
+
+    def replay_all(calibs):
+        for l, c in enumerate(calibs):
+            c.freeze_replay(w.k_pool[l], w.v_pool[l])
+
+    def write_all(calibs):
+        for l, c in enumerate(calibs):
+            k, v, s, kp, vp = chunks(l)
+            fp8q.fp8_kv_write(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:], kp, vp, scale_dev=c.scale_dev)
+
+    phases = [("observe_stage_write", stage_all), ("amax", observe_all),
+              ("freeze_replay", replay_all), ("kv_write", write_all)]
+    seqs = [("group_quant", [], lambda c: fp8q.fp8_group_quant(w.x, w.q, w.s), 1)]
+    for i, (label, fn) in enumerate(phases):
+        seqs.append((label, [f for _, f in phases[:i]], fn, L))
+    for label, prefix, body, n in seqs:
+        with torch.cuda.stream(stream):
+            w.states.copy_(w.states_init)
+            calibs = w.calibrators()
+            for f in prefix:
+                f(calibs)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        before = fp8q.launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            body(calibs)
+        assert fp8q.launch_count() - before == n, label
+        ts = time_graph(w, stream, g, reps, reset_state=False)
+        out[label] = (1e3 * statistics.median(ts) / n, n)
+        del g
+        for c in calibs:
+            c.close()
+    return out
 
 
 def run_native(args, dist: Dist) -> dict | None:
@@ -290,30 +362,16 @@ def run_native(args, dist: Dist) -> dict | None:
     torch.cuda.synchronize()
     assert fp8q.fp8q_device_error(clear=True) == 0
 
-    graph, events, labels, launches, graph_calibs = capture(w, stream, with_events=True)
+    graph, labels, launches, graph_calibs = capture(w, stream)
     assert launches == len(labels), (launches, len(labels))
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     clocks = ClockSampler(smi_gpu_id(dist.local_rank)) if dist.rank == 0 else None
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            w.reset(i)
-            graph.replay()
+    time_graph(w, stream, graph, args.warmup, reset_state=True)
     torch.cuda.synchronize()
 
     dist.barrier()
     torch.cuda.synchronize()
-    step_ms, per_label = [], {l: [] for l in set(labels)}
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            w.reset(i)
-            start.record()
-            graph.replay()
-            end.record()
-            end.synchronize()
-            step_ms.append(start.elapsed_time(end))
-            for j, lab in enumerate(labels):
-                per_label[lab].append(events[j].elapsed_time(events[j + 1]))
+    step_ms = time_graph(w, stream, graph, args.steps, reset_state=True)
     torch.cuda.synchronize()
     dist.barrier()
     clock_info = clocks.stop() if clocks is not None else None
@@ -338,6 +396,7 @@ def run_native(args, dist: Dist) -> dict | None:
     assert fp8q.fp8q_device_error(clear=True) == 0
 
     # eager (no graph) step time through the Python binding, for context
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     eager_ms = []
     with torch.cuda.stream(stream):
         for i in range(min(args.steps, 20)):
@@ -349,6 +408,7 @@ def run_native(args, dist: Dist) -> dict | None:
             end.synchronize()
             eager_ms.append(start.elapsed_time(end))
 
+    seq = kernel_sequences(w, stream, reps=max(5, min(args.steps, 50)))
     targets = measure_targets(w, stream, args)
     e2e = None if args.no_e2e else measure_e2e(w, stream, args)
     del graph
@@ -358,15 +418,15 @@ def run_native(args, dist: Dist) -> dict | None:
     result = None
     if dist.rank == 0:
         kernels = {}
-        for lab, ts in per_label.items():
+        kernel_time = sum(us * labels.count(lab) for lab, (us, _) in seq.items())
+        for lab, (avg_us, _) in seq.items():
             n_per_step = labels.count(lab)
-            avg_us = 1e3 * sum(ts) / len(ts)
             b = launch_bytes(lab)
             gbs = b / (avg_us * 1e-6) / 1e9
             kernels[lab] = {"launches_per_step": n_per_step, "avg_us": round(avg_us, 3),
                             "bytes_per_launch": b, "gbs": round(gbs, 1),
                             "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                            "share_of_step": round(n_per_step * avg_us / (1e3 * statistics.mean(step_ms)), 4)}
+                            "share": round(n_per_step * avg_us / kernel_time, 4)}
         dominant = max(kernels, key=lambda k: kernels[k]["launches_per_step"] * kernels[k]["avg_us"])
         dk = kernels[dominant]
         ms = 1e3 * max_s / args.steps
@@ -383,8 +443,10 @@ def run_native(args, dist: Dist) -> dict | None:
                              f"{workloads.LARGE_NUM_BLOCKS}-block pools of 16, window "
                              f"{workloads.LARGE_WINDOW_REQUEST}->4096, chunks {CHUNK1}+{CHUNK2}: "
                              "stage+write, freeze, replay, crossing write)"),
-                "l2": "flushed before every step (2x L2 write, untimed)",
-                "timing": "CUDA graph replay of the step's 65 launches; CUDA events",
+                "l2": "flushed before every step (2x L2 write, then 2x L2 read; untimed)",
+                "timing": ("CUDA graph replay of the step's 65 launches (programmatic "
+                           "dependent launch), CUDA events around each step; per-kernel "
+                           "times from graphs of each kernel's launches in step order"),
                 "bytes_per_step": step_bytes(args.layers),
                 "parallelism": f"replicas x{dist.world} (one step per GPU, no collective)",
             },
@@ -420,23 +482,15 @@ def measure_targets(w: Workload, stream, args) -> dict:
     reps = max(3, min(args.steps, 50))
 
     def timed(fn, n_launch):
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_launch + 1)]
         with torch.cuda.stream(stream):
             fn(lambda i: None)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            evs[0].record()
-            fn(lambda i: evs[i + 1].record())
-        times = []
-        with torch.cuda.stream(stream):
-            for i in range(reps):
-                w.flush_buf.fill_(i & 0xFF)
-                g.replay()
-                torch.cuda.synchronize()
-                times += [evs[j].elapsed_time(evs[j + 1]) for j in range(n_launch)]
+            fn(lambda i: None)
+        ts = time_graph(w, stream, g, reps, reset_state=False)
         del g
-        return statistics.mean(times) * 1e3
+        return statistics.median(ts) * 1e3 / n_launch
 
     def gq(mark):
         fp8q.fp8_group_quant(w.x, w.q, w.s)
@@ -621,6 +675,22 @@ def run_reference(args) -> dict | None:
     }
 
 
+def run_profile(args) -> None:
+    """A few eager steps on `--layers` layers, for an ncu capture of one kernel
+    (select it with ncu -k / -s / -c).  Prints nothing measured."""
+    torch.cuda.set_device(0)
+    w = Workload(torch.device("cuda", 0), args.layers)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup + args.steps):
+            w.reset(i)
+            w.issue(w.calibrators(), lambda _l: None)
+    torch.cuda.synchronize()
+    assert w.fp8q.fp8q_device_error(clear=True) == 0
+    print(json.dumps({"profile": "done", "layers": args.layers,
+                      "steps": args.warmup + args.steps}))
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -631,6 +701,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="run a few eager steps for an ncu capture and exit")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -641,6 +713,9 @@ def parse_args(argv=None):
 
 def main(argv=None) -> int:
     args = parse_args(argv)
+    if args.profile:
+        run_profile(args)
+        return 0
     if args.impl == "reference":
         res = run_reference(args)
     else:

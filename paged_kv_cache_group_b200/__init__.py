@@ -41,16 +41,19 @@ def _ptr(t) -> int:
 
 
 def _bf16_rows(t: torch.Tensor, name: str):
-    """[T, ...] bf16 with contiguous rows; returns (rows, row stride, E)."""
+    """``[T, ...]`` bf16 whose rows (all dimensions after the first) are
+    contiguous; returns (rows, row stride in elements, elements per row)."""
     if t.dtype != torch.bfloat16 or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+    if t.dim() < 2:
+        raise ValueError(f"{name} must have a row dimension and at least one more")
     rows = t.shape[0]
-    flat = t.reshape(rows, -1) if t.dim() > 2 else t
-    if flat.dim() != 2 or (flat.shape[1] > 1 and flat.stride(1) != 1):
-        raise ValueError(f"{name} rows must be contiguous")
-    if t.dim() > 2 and flat.data_ptr() != t.data_ptr():
-        raise ValueError(f"{name} rows must be contiguous")
-    return rows, flat.stride(0), flat.shape[1]
+    inner = 1
+    for size, stride in zip(reversed(t.shape[1:]), reversed(t.stride()[1:])):
+        if size != 1 and stride != inner:
+            raise ValueError(f"{name} rows must be contiguous")
+        inner *= size
+    return rows, (t.stride(0) if rows > 1 else inner), inner
 
 
 # ---------------------------------------------------------------------------

@@ -47,6 +47,13 @@ bool valid_rows(const void *k, const void *v, int64_t key_stride, int64_t value_
     return true;
 }
 
+int32_t pow2_shift(int32_t v) {
+    if (v <= 0 || (v & (v - 1)) != 0) return -1;
+    int32_t s = 0;
+    while ((1 << s) != v) ++s;
+    return s;
+}
+
 bool valid_pools(const void *k_pool, const void *v_pool, int32_t block_size,
                  int64_t cache_stride, int64_t num_blocks, int64_t elems) {
     if (block_size <= 0 || num_blocks < 0) return false;
@@ -161,6 +168,7 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
     p.k_pool = static_cast<uint8_t *>(k_pool);
     p.v_pool = static_cast<uint8_t *>(v_pool);
     p.block_size = block_size;
+    p.block_shift = pow2_shift(block_size);
     p.cache_stride = cache_stride;
     p.num_slots = num_blocks * block_size;
     p.freeze_amax = amax_bits(c);
@@ -211,6 +219,7 @@ KvPass write_pass(const void *k, const void *v, int64_t key_stride, int64_t valu
     p.k_pool = static_cast<uint8_t *>(k_pool);
     p.v_pool = static_cast<uint8_t *>(v_pool);
     p.block_size = block_size;
+    p.block_shift = pow2_shift(block_size);
     p.cache_stride = cache_stride;
     p.num_slots = num_blocks * block_size;
     p.do_write = true;
@@ -384,6 +393,7 @@ FP8Q_API fp8q_status fp8_kv_calib_observe_write(
         p.k_pool = w.k_pool;
         p.v_pool = w.v_pool;
         p.block_size = block_size;
+        p.block_shift = w.block_shift;
         p.cache_stride = cache_stride;
         p.num_slots = w.num_slots;
         p.k_scale = FP8Q_PROVISIONAL_SCALE;

@@ -27,6 +27,7 @@ struct KvPass {
     uint8_t *k_pool = nullptr;
     uint8_t *v_pool = nullptr;
     int32_t block_size = 0;
+    int32_t block_shift = -1;   // log2(block_size) when it is a power of two
     int64_t cache_stride = 0;
     int64_t num_slots = 0;
     // Scale source, first match wins:
