@@ -58,6 +58,7 @@ typedef int32_t fp8q_status;
 #define FP8Q_ECUDA (-2)       /* a CUDA call failed                          */
 #define FP8Q_ESTATE (-3)      /* calibration call out of order               */
 #define FP8Q_ENOMEM (-4)      /* host memory for a handle could not be had   */
+#define FP8Q_ETOOBIG (-5)     /* needs more than the library's fixed scratch */
 
 /* Bits of the sticky per-device error word. */
 #define FP8Q_DEVERR_SLOT_OUT_OF_RANGE 0x1u  /* slot >= num_blocks*block_size: token skipped */
@@ -197,6 +198,9 @@ FP8Q_API fp8q_status fp8_kv_amax_observe(const void *k, const void *v,
 
 /* Opaque per-layer calibrator (host memory, owned by the library). */
 typedef struct fp8_kv_calib fp8_kv_calib;
+
+/* Size of the fixed device scratch array behind fp8_kv_calib_window_noalloc. */
+#define FP8Q_NOALLOC_SCRATCH_BYTES (1 << 20)
 
 /* Step reported by an observe. */
 #define FP8Q_STEP_STAGE 1           /* in the window, batch staged           */
@@ -367,6 +371,60 @@ FP8Q_API fp8q_status fp8_kv_calib_read_state(const fp8_kv_calib *calib,
 
 /* Frees the host handle (no device memory is owned). NULL is ignored. */
 FP8Q_API void fp8_kv_calib_destroy(fp8_kv_calib *calib);
+
+/*
+ * fp8_kv_calib_window_noalloc -- one layer's calibration window in one call,
+ * for callers that cannot allocate device memory.
+ *
+ * The source pages have no counterpart of this call: their calibrator
+ * allocates its staging on first use.  Some callers cannot do that -- an
+ * engine that gives all device memory to its KV pool at start-up and
+ * forbids later cudaMalloc, code that must not risk the device-wide
+ * synchronization an allocation or free can cause, a host that gives the
+ * library no allocator.  This call needs no device memory from anyone: its
+ * scratch (the window's staged bf16 K/V rows and slots, and the 16-byte
+ * calibration state) is a fixed array of FP8Q_NOALLOC_SCRATCH_BYTES inside
+ * the library, which every device that loads the library holds until the
+ * process exits.  The call allocates nothing, host or device.
+ *
+ * Result: exactly what a calibrator made by fp8_kv_calib_create(window_tokens,
+ * headroom, ...) with staging for the whole window produces when it is fed
+ * the batches in order through fp8_kv_calib_observe_write: batches before the
+ * one that reaches the window are written at the provisional scale (and
+ * staged), that batch's arrival freezes the scales and replays the staged
+ * batches in order, and it and every later batch are written at the frozen
+ * scales.  If the batches end before the window is reached nothing is frozen
+ * or replayed (the staging does not outlive the call).
+ *
+ *   k, v, key_stride, value_stride, slot_mapping
+ *                  all batches' rows, one after another (batch b starts at
+ *                  the row after batch b-1's last), as for fp8_kv_write
+ *   batch_tokens   HOST int64 [num_batches], tokens of each batch (>= 0)
+ *   num_batches    >= 0
+ *   num_kv_heads, head_dim, window_tokens, headroom
+ *                  as for fp8_kv_calib_create (clamps included)
+ *   k_pool, v_pool, block_size, cache_stride, num_blocks
+ *                  the layer's pools, as for fp8_kv_write
+ *   scales_out     optional device fp32 [2]: receives {k_scale, v_scale}
+ *                  after the last batch (2.0 if the window was not reached)
+ * Limit: the rows staged before the freeze need staged * (4 * E + 8) bytes,
+ * E = num_kv_heads * head_dim; more than FP8Q_NOALLOC_SCRATCH_BYTES - 256
+ * returns FP8Q_ETOOBIG before anything is enqueued.  At most window - 1 rows
+ * are ever staged, so with 4 x 128 rows every window of up to 510 tokens fits.
+ * Sharing: every call uses the same array and leaves its contents there;
+ * the call initialises what must start from zero.  Calls whose work overlaps
+ * on the GPU (two streams, two threads) race on the array: serialize them.
+ * Set-up: the first call on each device looks up the array's device address
+ * (with that device current) and caches it; make that first call before any
+ * stream capture.
+ * Returns FP8Q_OK, FP8Q_EINVAL, FP8Q_ETOOBIG, FP8Q_ECUDA.
+ */
+FP8Q_API fp8q_status fp8_kv_calib_window_noalloc(
+    const void *k, const void *v, int64_t key_stride, int64_t value_stride,
+    const int64_t *slot_mapping, const int64_t *batch_tokens, int32_t num_batches,
+    int32_t num_kv_heads, int32_t head_dim, int64_t window_tokens, float headroom,
+    void *k_pool, void *v_pool, int32_t block_size, int64_t cache_stride,
+    int64_t num_blocks, float *scales_out, void *stream);
 
 /*
  * fp8_kv_graphs_ready -- whether CUDA graphs may be captured again.

@@ -231,6 +231,29 @@ class KvCalibration:
         return tuple(out)
 
 
+def fp8_kv_calib_window_noalloc(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                                batch_tokens, window_tokens: int, headroom: float,
+                                k_pool: torch.Tensor, v_pool: torch.Tensor,
+                                scales_out: torch.Tensor | None = None, stream=None) -> None:
+    """One layer's calibration window in one call, with no device memory from
+    the caller or the library's user: the scratch is a fixed array inside the
+    library (see include/fp8q.h).  ``k``/``v`` hold every batch's rows back to
+    back; ``batch_tokens`` lists each batch's token count."""
+    t, ks, e = _bf16_rows(k, "k")
+    _, vs, _ = _bf16_rows(v, "v")
+    counts = [int(n) for n in batch_tokens]
+    if sum(counts) != t:
+        raise ValueError("batch_tokens must add up to the rows of k and v")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() < t:
+        raise ValueError("slot_mapping must be int64 with one entry per token")
+    nb, bs, cs = _pool_geometry(k_pool, v_pool, e)
+    arr = (ctypes.c_int64 * max(len(counts), 1))(*counts)
+    _check("fp8_kv_calib_window_noalloc", lib.fp8_kv_calib_window_noalloc(
+        _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), arr, len(counts), k.shape[1], k.shape[2],
+        int(window_tokens), float(headroom), _ptr(k_pool), _ptr(v_pool), bs, cs, nb,
+        _ptr(scales_out), _stream(stream)))
+
+
 def fp8q_device_error(clear: bool = True) -> int:
     """Sticky device error bits of the current device (synchronizes)."""
     bits = ctypes.c_uint32()

@@ -54,18 +54,21 @@ SIGNATURES = {
     "fp8_kv_calib_read_state": (STATUS, [_P, _P, c.POINTER(_F)]),
     "fp8_kv_calib_destroy": (None, [_P]),
     "fp8_kv_graphs_ready": (_I32, [_P, _I64]),
+    "fp8_kv_calib_window_noalloc": (STATUS, [_P, _P, _I64, _I64, _P, _P, _I32, _I32, _I32, _I64,
+                                             _F, _P, _P, _I32, _I64, _I64, _P, _P]),
     "fp8q_device_error": (STATUS, [c.POINTER(c.c_uint32), _I32]),
     "fp8q_status_string": (c.c_char_p, [STATUS]),
     "fp8q_version": (_I32, []),
     "fp8q_launch_count": (_I64, []),
 }
 
-OK, EINVAL, ECUDA, ESTATE, ENOMEM = 0, -1, -2, -3, -4
+OK, EINVAL, ECUDA, ESTATE, ENOMEM, ETOOBIG = 0, -1, -2, -3, -4, -5
 STEP_STAGE, STEP_STAGE_DECLINED, STEP_FREEZE, STEP_FROZEN = 1, 2, 3, 4
 DEVERR_SLOT_OUT_OF_RANGE, DEVERR_BAD_SCALE = 0x1, 0x2
 MAX_STAGED_TOKENS = 4096
 PROVISIONAL_SCALE = 2.0
 CALIB_STATE_BYTES = 16
+NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class Fp8qError(RuntimeError):

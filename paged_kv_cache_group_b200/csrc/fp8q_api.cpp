@@ -459,6 +459,7 @@ FP8Q_API const char *fp8q_status_string(fp8q_status status) {
     case FP8Q_ECUDA: return "CUDA error";
     case FP8Q_ESTATE: return "calibration call out of order";
     case FP8Q_ENOMEM: return "out of host memory";
+    case FP8Q_ETOOBIG: return "request exceeds the fixed scratch of the allocation-free call";
     default: return "unknown status";
     }
 }
