@@ -5,11 +5,12 @@ One step is one 4593-token prefill through every operation of the path:
   * fp8_group_quant of the 4593 x 5120 bf16 activation (1x128 groups);
   * for each of 16 layers (4 KV heads x 128 dims, 8192-block pools of 16
     slots), the calibrating KV write of that layer's 4593 tokens, arriving in
-    two chunks: 4095 tokens inside the window (one fused pass: absmax, staging
-    copy, provisional-scale write), then 498 tokens that reach the 4096-token
-    window (absmax; freeze and replay of the 4095 staged tokens; write of the
+    two chunks through fp8_kv_calib_observe_write: 4095 tokens inside the
+    window (one fused pass: absmax, staging copy, provisional-scale write),
+    then 498 tokens that reach the 4096-token window (absmax, then one launch
+    that freezes the scales, replays the 4095 staged tokens and writes the
     crossing chunk at the frozen scale).
-That is 1 + 16 x 4 = 65 kernel launches, issued through the C ABI and
+That is 1 + 16 x 3 = 49 kernel launches, issued through the C ABI and
 replayed as one CUDA graph.  Before every step L2 is flushed (a 2x-L2 write,
 then a 2x-L2 read of a clean buffer) and the calibrators' device state is
 reset, both outside the timed region.
@@ -54,23 +55,23 @@ M, K = workloads.PREFILL_M, workloads.PREFILL_K
 PER_TOKEN = {
     "observe_stage_write": 2 * E * 2 + 8 + 2 * E + 2 * E * 2 + 8,   # 5136
     "amax": 2 * E * 2,                                             # 2048
-    "freeze_replay": 2 * E * 2 + 8 + 2 * E,                        # 3080
+    "replay_crossing": 2 * E * 2 + 8 + 2 * E,                      # 3080, staged and crossing
     "kv_write": 2 * E * 2 + 8 + 2 * E,                             # 3080
 }
+STEP_KERNELS = ("observe_stage_write", "amax", "replay_crossing")
 GROUP_QUANT_BYTES = M * K * 3 + M * (K // 128) * 4                 # 71,283,360
 
 
 def launch_bytes(label: str) -> int:
     if label == "group_quant":
         return GROUP_QUANT_BYTES
-    tokens = {"observe_stage_write": CHUNK1, "amax": CHUNK2, "freeze_replay": CHUNK1,
-              "kv_write": CHUNK2}[label]
+    tokens = {"observe_stage_write": CHUNK1, "amax": CHUNK2, "replay_crossing": CHUNK1 + CHUNK2,
+              "kv_write": TOKENS}[label]
     return PER_TOKEN[label] * tokens
 
 
 def step_bytes(layers: int) -> int:
-    per_layer = sum(launch_bytes(k) for k in ("observe_stage_write", "amax", "freeze_replay",
-                                              "kv_write"))
+    per_layer = sum(launch_bytes(k) for k in STEP_KERNELS)
     return GROUP_QUANT_BYTES + layers * per_layer
 
 
@@ -233,28 +234,20 @@ class Workload:
         self.states.copy_(self.states_init)
         self.flush(i)
 
-    def issue(self, calibs, mark) -> None:
+    def issue(self, calibs) -> None:
         fp8q = self.fp8q
         fp8q.fp8_group_quant(self.x, self.q, self.s)
-        mark("group_quant")
         for l, c in enumerate(calibs):
             k, v, s = self.k[l], self.v[l], self.slots[l]
             kp, vp = self.k_pool[l], self.v_pool[l]
             st = c.observe_write(k[:CHUNK1], v[:CHUNK1], s[:CHUNK1], kp, vp)
             assert st == fp8q.STEP_STAGE, st
-            mark("observe_stage_write")
-            st = c.observe(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:])
+            st = c.observe_write(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:], kp, vp)
             assert st == fp8q.STEP_FREEZE, st
-            mark("amax")
-            n = c.freeze_replay(kp, vp)
-            assert n == CHUNK1, n
-            mark("freeze_replay")
-            fp8q.fp8_kv_write(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:], kp, vp, scale_dev=c.scale_dev)
-            mark("kv_write")
 
 
 def labels_of(layers: int) -> list[str]:
-    return ["group_quant"] + ["observe_stage_write", "amax", "freeze_replay", "kv_write"] * layers
+    return ["group_quant"] + list(STEP_KERNELS) * layers
 
 
 def capture(w: Workload, stream):
@@ -267,7 +260,7 @@ def capture(w: Workload, stream):
     graph = torch.cuda.CUDAGraph()
     before = w.fp8q.launch_count()
     with torch.cuda.graph(graph, stream=stream):
-        w.issue(calibs, lambda _l: None)
+        w.issue(calibs)
     launches = w.fp8q.launch_count() - before
     # The graph writes into these calibrators' staging tensors on every
     # replay: the caller keeps them alive as long as the graph.
@@ -294,39 +287,28 @@ def time_graph(w: Workload, stream, graph, reps: int, reset_state: bool) -> list
 def kernel_sequences(w: Workload, stream, reps: int) -> dict:
     """Average launch duration of each kernel of the step, from a graph of its
     launches exactly as the step issues them (one per layer, back to back),
-    the state before them prepared eagerly.  Returns {label: (us, launches)}."""
+    the state before them prepared eagerly.  The merged freeze launch is only
+    reachable together with the crossing chunk's absmax, so its time is the
+    difference between that pair's graph and the absmax-only graph.
+    Returns {label: (us per launch, launches per graph)}."""
     fp8q = w.fp8q
     L = w.layers
-    out = {}
-
-    def chunks(l):
-        return (w.k[l], w.v[l], w.slots[l], w.k_pool[l], w.v_pool[l])
 
     def stage_all(calibs):
         for l, c in enumerate(calibs):
-            k, v, s, kp, vp = chunks(l)
-            c.observe_write(k[:CHUNK1], v[:CHUNK1], s[:CHUNK1], kp, vp)
+            c.observe_write(w.k[l][:CHUNK1], w.v[l][:CHUNK1], w.slots[l][:CHUNK1],
+                            w.k_pool[l], w.v_pool[l])
 
-    def observe_all(calibs):
+    def amax_all(calibs):
         for l, c in enumerate(calibs):
-            k, v, s, _, _ = chunks(l)
-            c.observe(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:])
+            c.observe(w.k[l][CHUNK1:], w.v[l][CHUNK1:], w.slots[l][CHUNK1:])
 
-    def replay_all(calibs):
+    def freeze_all(calibs):
         for l, c in enumerate(calibs):
-            c.freeze_replay(w.k_pool[l], w.v_pool[l])
+            c.observe_write(w.k[l][CHUNK1:], w.v[l][CHUNK1:], w.slots[l][CHUNK1:],
+                            w.k_pool[l], w.v_pool[l])
 
-    def write_all(calibs):
-        for l, c in enumerate(calibs):
-            k, v, s, kp, vp = chunks(l)
-            fp8q.fp8_kv_write(k[CHUNK1:], v[CHUNK1:], s[CHUNK1:], kp, vp, scale_dev=c.scale_dev)
-
-    phases = [("observe_stage_write", stage_all), ("amax", observe_all),
-              ("freeze_replay", replay_all), ("kv_write", write_all)]
-    seqs = [("group_quant", [], lambda c: fp8q.fp8_group_quant(w.x, w.q, w.s), 1)]
-    for i, (label, fn) in enumerate(phases):
-        seqs.append((label, [f for _, f in phases[:i]], fn, L))
-    for label, prefix, body, n in seqs:
+    def timed(prefix, body, n):
         with torch.cuda.stream(stream):
             w.states.copy_(w.states_init)
             calibs = w.calibrators()
@@ -337,13 +319,19 @@ def kernel_sequences(w: Workload, stream, reps: int) -> dict:
         before = fp8q.launch_count()
         with torch.cuda.graph(g, stream=stream):
             body(calibs)
-        assert fp8q.launch_count() - before == n, label
+        assert fp8q.launch_count() - before == n
         ts = time_graph(w, stream, g, reps, reset_state=False)
-        out[label] = (1e3 * statistics.median(ts) / n, n)
         del g
         for c in calibs:
             c.close()
-    return out
+        return 1e3 * statistics.mean(ts)
+
+    gq = timed([], lambda c: fp8q.fp8_group_quant(w.x, w.q, w.s), 1)
+    stage = timed([], stage_all, L)
+    amax = timed([stage_all], amax_all, L)
+    pair = timed([stage_all], freeze_all, 2 * L)
+    return {"group_quant": (gq, 1), "observe_stage_write": (stage / L, L),
+            "amax": (amax / L, L), "replay_crossing": (max(pair - amax, 0.0) / L, L)}
 
 
 def run_native(args, dist: Dist) -> dict | None:
@@ -358,7 +346,7 @@ def run_native(args, dist: Dist) -> dict | None:
     with torch.cuda.stream(stream):
         for i in range(2):
             w.reset(i)
-            w.issue(w.calibrators(), lambda _l: None)
+            w.issue(w.calibrators())
     torch.cuda.synchronize()
     assert fp8q.fp8q_device_error(clear=True) == 0
 
@@ -388,7 +376,7 @@ def run_native(args, dist: Dist) -> dict | None:
     pools_graph = (w.k_pool[-1].clone(), w.v_pool[-1].clone())
     with torch.cuda.stream(stream):
         w.reset(0)
-        w.issue(w.calibrators(), lambda _l: None)
+        w.issue(w.calibrators())
     torch.cuda.synchronize()
     assert torch.equal(q_graph, w.q)
     assert torch.equal(pools_graph[0], w.k_pool[-1]) and torch.equal(pools_graph[1], w.v_pool[-1])
@@ -403,7 +391,7 @@ def run_native(args, dist: Dist) -> dict | None:
             calibs = w.calibrators()
             w.reset(i)
             start.record()
-            w.issue(calibs, lambda _l: None)
+            w.issue(calibs)
             end.record()
             end.synchronize()
             eager_ms.append(start.elapsed_time(end))
@@ -442,9 +430,9 @@ def run_native(args, dist: Dist) -> dict | None:
                              f"({workloads.KV_HEADS} KV heads x {workloads.HEAD_DIM}, "
                              f"{workloads.LARGE_NUM_BLOCKS}-block pools of 16, window "
                              f"{workloads.LARGE_WINDOW_REQUEST}->4096, chunks {CHUNK1}+{CHUNK2}: "
-                             "stage+write, freeze, replay, crossing write)"),
+                             "stage+write; absmax; freeze+replay+crossing write)"),
                 "l2": "flushed before every step (2x L2 write, then 2x L2 read; untimed)",
-                "timing": ("CUDA graph replay of the step's 65 launches (programmatic "
+                "timing": ("CUDA graph replay of the step's 49 launches (programmatic "
                            "dependent launch), CUDA events around each step; per-kernel "
                            "times from graphs of each kernel's launches in step order"),
                 "bytes_per_step": step_bytes(args.layers),
@@ -490,7 +478,7 @@ def measure_targets(w: Workload, stream, args) -> dict:
             fn(lambda i: None)
         ts = time_graph(w, stream, g, reps, reset_state=False)
         del g
-        return statistics.median(ts) * 1e3 / n_launch
+        return statistics.mean(ts) * 1e3 / n_launch
 
     def gq(mark):
         fp8q.fp8_group_quant(w.x, w.q, w.s)
@@ -545,7 +533,7 @@ def measure_e2e(w: Workload, stream, args) -> dict:
                 w.k[l].view(TOKENS, E).copy_(hk[l], non_blocking=True)
                 w.v[l].view(TOKENS, E).copy_(hv[l], non_blocking=True)
                 w.slots[l].copy_(hs[l], non_blocking=True)
-            w.issue(calibs, lambda _l: None)
+            w.issue(calibs)
             oq.copy_(w.q, non_blocking=True)
             os_.copy_(w.s, non_blocking=True)
             ost.copy_(w.states, non_blocking=True)
@@ -610,8 +598,7 @@ def reference_sample():
 
 def sample_bytes() -> int:
     gq = SAMPLE_ROWS * K * 3 + SAMPLE_ROWS * (K // 128) * 4
-    per_layer = sum(launch_bytes(k) for k in ("observe_stage_write", "amax", "freeze_replay",
-                                              "kv_write"))
+    per_layer = sum(launch_bytes(k) for k in STEP_KERNELS)
     return gq + SAMPLE_LAYERS * per_layer
 
 
@@ -675,6 +662,106 @@ def run_reference(args) -> dict | None:
     }
 
 
+def run_sweep(args) -> list[dict]:
+    """Decode-width sweep: group quant at M in {1,2,4,8,16} x K in {5120,16384},
+    1000 back-to-back launches per shape, timed as plain stream launches
+    through the binding and as a CUDA graph of 1000 launches.  Launch-bound by
+    design; inputs stay in L2, as they do in a decode loop."""
+    import paged_kv_cache_group_b200 as fp8q
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream()
+    n = 1000
+    out = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for m in workloads.DECODE_MS:
+        for k in workloads.DECODE_KS:
+            bits = workloads.decode_quant(m, k)
+            x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+            q = torch.empty((m, k), dtype=torch.uint8, device=dev)
+            sc = torch.empty((m, k // 128), dtype=torch.float32, device=dev)
+            with torch.cuda.stream(stream):
+                for _ in range(20):
+                    fp8q.fp8_group_quant(x, q, sc)
+                torch.cuda.synchronize()
+                plain = []
+                for _ in range(3):
+                    start.record()
+                    for _ in range(n):
+                        fp8q.fp8_group_quant(x, q, sc)
+                    end.record()
+                    end.synchronize()
+                    plain.append(start.elapsed_time(end) * 1e3 / n)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    fp8q.fp8_group_quant(x, q, sc)
+            graph = []
+            with torch.cuda.stream(stream):
+                for _ in range(5):
+                    start.record()
+                    g.replay()
+                    end.record()
+                    end.synchronize()
+                    graph.append(start.elapsed_time(end) * 1e3 / n)
+            del g
+            b = m * k * 3 + m * (k // 128) * 4
+            us_p, us_g = statistics.median(plain), statistics.median(graph)
+            out.append({"m": m, "k": k, "bytes": b, "plain_us_per_launch": round(us_p, 3),
+                        "graph_us_per_launch": round(us_g, 3),
+                        "graph_gbs": round(b / (us_g * 1e-6) / 1e9, 1),
+                        "graph_tokens_per_s": round(m / (us_g * 1e-6), 1)})
+    return out
+
+
+def run_calib(args) -> dict:
+    """The 256-token calibration window of one layer (13 + 32-token batches,
+    freeze at batch 9, two batches after it) through fp8_kv_calib_observe_write,
+    eager, with L2 flushed before each window; CUDA events around the window."""
+    import paged_kv_cache_group_b200 as fp8q
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    spec, batches, _ = workloads.calib_window()
+    def rows(bits):
+        t = bits.shape[0]
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev).view(t, 4, 128)
+    ks = [rows(b.k) for b in batches]
+    vs = [rows(b.v) for b in batches]
+    ss = [torch.from_numpy(b.slot_mapping).to(dev) for b in batches]
+    shape = (spec.num_blocks, spec.block_size, spec.heads, spec.dim)
+    kp = torch.full(shape, workloads.SENTINEL, dtype=torch.uint8, device=dev)
+    vp = torch.full(shape, workloads.SENTINEL, dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(2 * l2, dtype=torch.uint8, device=dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.Stream()
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup + args.steps):
+            cal = fp8q.KvCalibration(workloads.CALIB_WINDOW, 1.0, 4, 128, dev)
+            flush_w.fill_(i & 0xFF)
+            torch.amax(flush_r)
+            torch.cuda._sleep(1_000_000)       # let the host queue the window ahead
+            start.record()
+            for k, v, s in zip(ks, vs, ss):
+                cal.observe_write(k, v, s, kp, vp)
+            end.record()
+            end.synchronize()
+            if i >= args.warmup:
+                times.append(start.elapsed_time(end) * 1e3)
+            cal.close()
+    staged = sum(b.num_tokens for b in batches[:8])
+    seen = sum(b.num_tokens for b in batches)
+    bytes_ = (staged * PER_TOKEN["observe_stage_write"] + batches[8].num_tokens * 2048 +
+              (staged + batches[8].num_tokens) * 3080 +
+              sum(b.num_tokens for b in batches[9:]) * 3080)
+    us = statistics.median(times)
+    return {"workload": "calibration window: 256 tokens, 4 x 128, batches 13 + 10 x 32",
+            "us_per_window": round(us, 2), "tokens": seen, "bytes": bytes_,
+            "gbs": round(bytes_ / (us * 1e-6) / 1e9, 1), "windows": len(times)}
+
+
 def run_profile(args) -> None:
     """A few eager steps on `--layers` layers, for an ncu capture of one kernel
     (select it with ncu -k / -s / -c).  Prints nothing measured."""
@@ -684,7 +771,7 @@ def run_profile(args) -> None:
     with torch.cuda.stream(stream):
         for i in range(args.warmup + args.steps):
             w.reset(i)
-            w.issue(w.calibrators(), lambda _l: None)
+            w.issue(w.calibrators())
     torch.cuda.synchronize()
     assert w.fp8q.fp8q_device_error(clear=True) == 0
     print(json.dumps({"profile": "done", "layers": args.layers,
@@ -703,6 +790,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--profile", action="store_true",
                     help="run a few eager steps for an ncu capture and exit")
+    ap.add_argument("--sweep", action="store_true",
+                    help="decode-width sweep of the group quantizer (one JSON line per shape)")
+    ap.add_argument("--calib", action="store_true",
+                    help="time the 256-token calibration window end to end")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -715,6 +806,13 @@ def main(argv=None) -> int:
     args = parse_args(argv)
     if args.profile:
         run_profile(args)
+        return 0
+    if args.sweep:
+        for line in run_sweep(args):
+            print(json.dumps(line), flush=True)
+        return 0
+    if args.calib:
+        print(json.dumps(run_calib(args)), flush=True)
         return 0
     if args.impl == "reference":
         res = run_reference(args)

@@ -154,9 +154,16 @@ fp8q_status plan_observe(fp8_kv_calib *c, const void *k, const void *v, int64_t 
     return FP8Q_OK;
 }
 
+// The freeze's device work: every staged batch is rewritten, in the order it
+// was staged, at the scales frozen from the device maxima; the first launch
+// also publishes those scales to state_dev.  When `crossing` is given (the
+// batch that reached the window, as a write pass reading the published
+// scales) and fits in one launch with the last staged batch, the two share a
+// launch; otherwise the crossing batch is written by its own launch after the
+// replay.  Either way each slot ends with its last writer in arrival order.
 fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t block_size,
                        int64_t cache_stride, int64_t num_blocks, cudaStream_t stream,
-                       int64_t *replayed) {
+                       int64_t *replayed, const KvPass *crossing) {
     if (c->phase != kFreezePending) return FP8Q_ESTATE;
     if (!valid_pools(k_pool, v_pool, block_size, cache_stride, num_blocks, c->elems))
         return FP8Q_EINVAL;
@@ -174,32 +181,61 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
     p.freeze_amax = amax_bits(c);
     p.headroom = c->headroom;
     p.scale_out = scale_dev(c);
-    // The first launch also publishes the frozen scales (block 0 of that
-    // launch); with nothing staged a one-block launch does only that.  Empty
-    // staged batches after the first launch have nothing to rewrite.
+
+    // Last staged batch with rows: the one the crossing batch joins.
+    int64_t last = -1;
+    for (int64_t i = 0; i < static_cast<int64_t>(c->batches.size()); ++i)
+        if (c->batches[i].num_tokens > 0) last = i;
+    KvPass probe = p;
+    if (crossing != nullptr) {
+        probe.x_tokens = crossing->num_tokens;
+    }
+    const bool merge = crossing != nullptr && crossing->num_tokens > 0 &&
+                       crossing->elems == p.elems && fp8q::can_merge_crossing(probe);
+    auto with_crossing = [&](KvPass q) {
+        q.xk = crossing->k;
+        q.xv = crossing->v;
+        q.x_key_stride = crossing->key_stride;
+        q.x_value_stride = crossing->value_stride;
+        q.x_slots = crossing->slot_mapping;
+        q.x_tokens = crossing->num_tokens;
+        return q;
+    };
+
     int64_t rewritten = 0;
     bool published = false;
-    for (const StagedBatch &b : c->batches) {
-        if (b.num_tokens == 0 && published) continue;
-        p.k = c->stage_k + b.offset_tokens * c->elems;
-        p.v = c->stage_v + b.offset_tokens * c->elems;
-        p.slot_mapping = c->stage_slots + b.offset_tokens;
-        p.num_tokens = b.num_tokens;
-        cudaError_t e = fp8q::launch_kv_pass(p, stream);
-        if (e != cudaSuccess) return FP8Q_ECUDA;
-        rewritten += b.num_tokens;
+    if (merge && last < 0) {
+        // nothing staged with rows: the crossing batch alone, publishing the scales
+        KvPass q = with_crossing(p);
+        q.num_tokens = 0;
+        if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
         published = true;
-    }
-    if (!published) {
-        p.num_tokens = 0;
-        cudaError_t e = fp8q::launch_kv_pass(p, stream);
-        if (e != cudaSuccess) return FP8Q_ECUDA;
+    } else {
+        for (int64_t i = 0; i < static_cast<int64_t>(c->batches.size()); ++i) {
+            const StagedBatch &b = c->batches[i];
+            if (b.num_tokens == 0 && published) continue;
+            p.k = c->stage_k + b.offset_tokens * c->elems;
+            p.v = c->stage_v + b.offset_tokens * c->elems;
+            p.slot_mapping = c->stage_slots + b.offset_tokens;
+            p.num_tokens = b.num_tokens;
+            const KvPass q = (merge && i == last) ? with_crossing(p) : p;
+            if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
+            rewritten += b.num_tokens;
+            published = true;
+        }
+        if (!published) {
+            p.num_tokens = 0;
+            if (fp8q::launch_kv_pass(p, stream) != cudaSuccess) return FP8Q_ECUDA;
+        }
+        if (crossing != nullptr && !merge) {
+            if (fp8q::launch_kv_pass(*crossing, stream) != cudaSuccess) return FP8Q_ECUDA;
+        }
     }
     const int64_t batches = static_cast<int64_t>(c->batches.size());
     c->batches.clear();
     c->used_tokens = 0;
     c->replayed_tokens = rewritten;
-    c->replayed_batches = static_cast<int64_t>(batches);
+    c->replayed_batches = batches;
     c->phase = kFrozen;
     if (replayed) *replayed = rewritten;
     return FP8Q_OK;
@@ -355,7 +391,7 @@ FP8Q_API fp8q_status fp8_kv_freeze_replay(fp8_kv_calib *calib, void *k_pool, voi
                                           int64_t *replayed_tokens) {
     if (calib == nullptr) return FP8Q_EINVAL;
     return run_replay(calib, k_pool, v_pool, block_size, cache_stride, num_blocks,
-                      as_stream(stream), replayed_tokens);
+                      as_stream(stream), replayed_tokens, nullptr);
 }
 
 FP8Q_API fp8q_status fp8_kv_calib_observe_write(
@@ -400,13 +436,13 @@ FP8Q_API fp8q_status fp8_kv_calib_observe_write(
         p.v_scale = FP8Q_PROVISIONAL_SCALE;
         return from_cuda(fp8q::launch_kv_pass(p, s));
     }
-    // FREEZE: the maxima must include this batch before any write
+    // FREEZE: the maxima must include this batch before any write; then the
+    // replay, with the crossing batch written at the frozen scales last
     cudaError_t e = fp8q::launch_kv_pass(p, s);
     if (e != cudaSuccess) return FP8Q_ECUDA;
-    st = run_replay(calib, k_pool, v_pool, block_size, cache_stride, num_blocks, s, nullptr);
-    if (st != FP8Q_OK) return st;
     w.scale_dev = scale_dev(calib);
-    return from_cuda(fp8q::launch_kv_pass(w, s));
+    return run_replay(calib, k_pool, v_pool, block_size, cache_stride, num_blocks, s, nullptr,
+                      &w);
 }
 
 FP8Q_API const float *fp8_kv_calib_scale_dev(const fp8_kv_calib *calib) {

@@ -42,6 +42,18 @@ struct KvPass {
     float k_scale = 1.0f;
     float v_scale = 1.0f;
 
+    // Crossing batch written by the same launch after a replayed staged
+    // batch (write passes only): tokens [num_tokens, num_tokens + x_tokens)
+    // come from xk / xv / x_slots.  A staged token whose slot the crossing
+    // batch also writes is skipped, so the crossing token is the last writer,
+    // as if the two had been written by two launches in that order.
+    const uint16_t *xk = nullptr;
+    const uint16_t *xv = nullptr;
+    int64_t x_key_stride = 0;
+    int64_t x_value_stride = 0;
+    const int64_t *x_slots = nullptr;
+    int64_t x_tokens = 0;
+
     // amax
     uint32_t *amax_bits = nullptr;
 
@@ -62,6 +74,11 @@ cudaError_t launch_group_quant(const uint16_t *x, int64_t x_row_stride, uint8_t 
 // Launches one KV pass.  A pass with no tokens still launches when it must
 // publish a frozen scale (freeze_amax and scale_out set).
 cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream);
+
+// Largest crossing batch a single launch can merge with a replay (its slots
+// go into a hash set in shared memory); larger ones use two launches.
+constexpr int64_t kMaxMergedCrossing = 8192;
+bool can_merge_crossing(const KvPass &p);
 
 // Enqueues state_dev = {0, 0, 2.0, 2.0} (bit patterns of the fp32 values).
 cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream);

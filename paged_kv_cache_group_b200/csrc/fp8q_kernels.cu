@@ -26,6 +26,7 @@
 #include <cstdint>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "fp8q_internal.h"
@@ -71,6 +72,17 @@ __device__ __forceinline__ void wait_for_previous_grid() {
 }
 __device__ __forceinline__ void allow_next_grid() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Warm L2 with bytes this thread is about to read.  Issued before
+// wait_for_previous_grid(), so the DRAM reads overlap the previous kernel's
+// tail.  It is only a hint: L2 is where the GPU's writes become coherent, so
+// a later load still returns whatever the previous kernel wrote.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
 }
 
 // Per-half max of |a| and |b| for two bf16x2 words (the sign bits of the
@@ -213,25 +225,27 @@ __global__ void __launch_bounds__(kGqThreads)
 group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
                    uint8_t *__restrict__ q, float *__restrict__ scales,
                    int64_t total_groups, uint32_t groups_per_row) {
-    wait_for_previous_grid();
-    allow_next_grid();
     const int lane = threadIdx.x & 31;
     const int sub = lane >> 2;   // group within the warp's eight
     const int ql = lane & 3;     // lane within the group
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kGqThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGqThreads) >> 5;
     const int64_t octets = (total_groups + 7) >> 3;
+    auto group_src = [&](int64_t g) -> const uint16_t * {
+        if (kPacked) return x + g * 128;
+        const uint64_t row = static_cast<uint64_t>(g) / groups_per_row;
+        return x + row * x_row_stride + (static_cast<uint64_t>(g) - row * groups_per_row) * 128;
+    };
+    // the first eight groups this warp reads: one 256-byte group per lane 0..7
+    if (lane < 8 && warp < octets && warp * 8 + lane < total_groups)
+        prefetch_l2_bulk(group_src(warp * 8 + lane), 256);
+    wait_for_previous_grid();
+    allow_next_grid();
 
     for (int64_t o = warp; o < octets; o += nwarps) {
         const int64_t g = o * 8 + sub;
         const bool valid = g < total_groups;
-        const uint16_t *src;
-        if (kPacked) {
-            src = x + g * 128;
-        } else {
-            const uint64_t row = static_cast<uint64_t>(g) / groups_per_row;
-            src = x + row * x_row_stride + (static_cast<uint64_t>(g) - row * groups_per_row) * 128;
-        }
+        const uint16_t *src = group_src(valid ? g : 0);
         uint4 c[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -270,77 +284,173 @@ group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
 // is one contiguous run (512 B of bf16 in, 256 B of codes out).  The slot
 // decides where the codes land: one token's entry is E contiguous bytes of the
 // pool, written as 32 8-byte stores per instruction.
+//
+// Each warp issues its first token's loads before anything else.  The scales
+// (a dependent load, and for a freeze an IEEE division and a reciprocal) are
+// resolved once per CTA by thread 0 while those loads are in flight, and
+// shared through shared memory.
 
 constexpr int kKvThreads = 256;
 constexpr int kKvWarps = kKvThreads / 32;
+constexpr uint32_t kEmptySlot = 0xFFFFFFFFu;
 
-// Scales of a write pass, resolved on the device (see KvPass).
-struct PassScales {
-    TensorEncoder k, v;
+// Shared-memory hash set of the crossing batch's slots (open addressing,
+// linear probing, 2^log2 entries, at most half full).
+__device__ __forceinline__ uint32_t slot_hash(uint32_t key, int log2) {
+    return (key * 2654435761u) >> (32 - log2);
+}
 
-    __device__ __forceinline__ void resolve(const KvPass &p) {
-        float ks, vs;
-        if (p.freeze_amax != nullptr) {
-            ks = freeze_scale(p.freeze_amax[0], p.headroom);
-            vs = freeze_scale(p.freeze_amax[1], p.headroom);
-            if (p.scale_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
-                p.scale_out[0] = ks;
-                p.scale_out[1] = vs;
-            }
-        } else if (p.scale_dev != nullptr) {
-            ks = p.scale_dev[0];
-            vs = p.scale_dev[1];
-        } else {
-            ks = p.k_scale;
-            vs = p.v_scale;
-        }
-        k.init(ks);
-        v.init(vs);
-        if (!(k.ok && v.ok) && blockIdx.x == 0 && threadIdx.x == 0)
-            atomicOr(&g_error_word, kErrScale);
+__device__ __forceinline__ void table_insert(uint32_t *tab, int log2, uint32_t key) {
+    const uint32_t mask = (1u << log2) - 1u;
+    uint32_t h = slot_hash(key, log2);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {   // bounded: the table is never full
+        const uint32_t prev = atomicCAS(&tab[h], kEmptySlot, key);
+        if (prev == kEmptySlot || prev == key) return;
+        h = (h + 1u) & mask;
     }
+}
+
+__device__ __forceinline__ bool table_contains(const uint32_t *tab, int log2, uint32_t key) {
+    const uint32_t mask = (1u << log2) - 1u;
+    uint32_t h = slot_hash(key, log2);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+        const uint32_t v = tab[h];
+        if (v == key) return true;
+        if (v == kEmptySlot) return false;
+        h = (h + 1u) & mask;
+    }
+    return false;
+}
+
+__device__ __forceinline__ int table_log2(int64_t entries) {
+    int log2 = 6;
+    while ((int64_t{1} << log2) < 2 * entries) ++log2;
+    return log2;
+}
+
+// Scales of a write pass (see KvPass), resolved by one thread.
+__device__ __forceinline__ void resolve_scales(const KvPass &p, TensorEncoder *enc) {
+    float ks, vs;
+    if (p.freeze_amax != nullptr) {
+        ks = freeze_scale(p.freeze_amax[0], p.headroom);
+        vs = freeze_scale(p.freeze_amax[1], p.headroom);
+        if (p.scale_out != nullptr && blockIdx.x == 0) {
+            p.scale_out[0] = ks;
+            p.scale_out[1] = vs;
+        }
+    } else if (p.scale_dev != nullptr) {
+        ks = p.scale_dev[0];
+        vs = p.scale_dev[1];
+    } else {
+        ks = p.k_scale;
+        vs = p.v_scale;
+    }
+    enc[0].init(ks);
+    enc[1].init(vs);
+    if (!(enc[0].ok && enc[1].ok) && blockIdx.x == 0) atomicOr(&g_error_word, kErrScale);
+}
+
+// A token's row pointers (staged or crossing) and its first 64 chunks.
+struct Row {
+    const uint16_t *k;
+    const uint16_t *v;
+    int64_t slot;
+    uint4 ka, kb, va, vb;
 };
+
+template <bool kCross, bool kSlot, int kChunks>
+__device__ __forceinline__ void load_row(const KvPass &p, int64_t t, int lane, int nchunks,
+                                         Row &r) {
+    if (kCross && t >= p.num_tokens) {
+        const int64_t u = t - p.num_tokens;
+        r.k = p.xk + u * p.x_key_stride;
+        r.v = p.xv + u * p.x_value_stride;
+        r.slot = __ldg(p.x_slots + u);
+    } else {
+        r.k = p.k + t * p.key_stride;
+        r.v = p.v + t * p.value_stride;
+        r.slot = kSlot ? __ldg(p.slot_mapping + t) : -1;
+    }
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const bool ha = lane < nchunks;
+    const bool hb = 32 + lane < nchunks;
+    r.ka = ha ? ld_once(r.k + lane * 8) : z;
+    r.kb = hb ? ld_once(r.k + (32 + lane) * 8) : z;
+    r.va = ha ? ld_once(r.v + lane * 8) : z;
+    r.vb = hb ? ld_once(r.v + (32 + lane) * 8) : z;
+}
 
 // kChunks: 16-byte chunks per row when fixed at compile time (64 for the
 // common 4 x 128 rows), or 0 for any multiple of 8 elements.
-template <bool kAmax, bool kStage, bool kWrite, int kChunks>
+template <bool kAmax, bool kStage, bool kWrite, bool kCross, int kChunks>
 __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) {
-    wait_for_previous_grid();
-    allow_next_grid();
+    extern __shared__ uint32_t s_table[];        // crossing slots (kCross)
+    __shared__ TensorEncoder s_enc[2];
 
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kKvThreads) >> 5;
     const int nchunks = kChunks > 0 ? kChunks : (p.elems >> 3);
-    const bool small_slots = p.num_slots <= 0x7FFFFFFF;
-    uint32_t kacc = 0, vacc = 0;
-    PassScales sc;
-    bool scales_ready = !kWrite;
+    const int64_t total = p.num_tokens + (kCross ? p.x_tokens : 0);
+    constexpr bool kSlot = kWrite || kStage;
 
-    for (int64_t t = warp; t < p.num_tokens; t += nwarps) {
-        // This token's loads go out first; the scales (a dependent load and
-        // an IEEE division) are resolved while they are in flight.
-        int64_t slot = -1;
-        if (kWrite || kStage) slot = __ldg(p.slot_mapping + t);
-        const uint16_t *krow = p.k + t * p.key_stride;
-        const uint16_t *vrow = p.v + t * p.value_stride;
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        const bool h0a = lane < nchunks;
-        const bool h0b = 32 + lane < nchunks;
-        uint4 ka = h0a ? ld_once(krow + lane * 8) : z;
-        uint4 kb = h0b ? ld_once(krow + (32 + lane) * 8) : z;
-        uint4 va = h0a ? ld_once(vrow + lane * 8) : z;
-        uint4 vb = h0b ? ld_once(vrow + (32 + lane) * 8) : z;
-        if (kWrite && !scales_ready) {
-            sc.resolve(p);
-            scales_ready = true;
+    // the first token's K row, V row and slot into L2 while the previous
+    // kernel finishes
+    if (warp < total && lane < 3) {
+        const bool crossing = kCross && warp >= p.num_tokens;
+        const int64_t u = warp - (crossing ? p.num_tokens : 0);
+        const uint32_t row_bytes = static_cast<uint32_t>(p.elems) * 2u;
+        if (lane == 0)
+            prefetch_l2_bulk(crossing ? p.xk + u * p.x_key_stride : p.k + u * p.key_stride, row_bytes);
+        else if (lane == 1)
+            prefetch_l2_bulk(crossing ? p.xv + u * p.x_value_stride : p.v + u * p.value_stride,
+                             row_bytes);
+        else if (kSlot)
+            prefetch_l2(crossing ? p.x_slots + u : p.slot_mapping + u);
+    }
+    wait_for_previous_grid();
+    allow_next_grid();
+
+    // 1. this warp's first token: loads out first
+    Row r;
+    int64_t t = warp;
+    if (t < total) load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
+
+    // 2. per CTA: the crossing slots' hash set, and the scales
+    int log2 = 0;
+    if (kCross) {
+        log2 = table_log2(p.x_tokens);
+        for (int i = threadIdx.x; i < (1 << log2); i += kKvThreads) s_table[i] = kEmptySlot;
+        __syncthreads();
+        for (int64_t i = threadIdx.x; i < p.x_tokens; i += kKvThreads) {
+            const int64_t s = __ldg(p.x_slots + i);
+            if (s >= 0 && s < p.num_slots) table_insert(s_table, log2, static_cast<uint32_t>(s));
         }
+    }
+    if (kWrite) {
+        if (threadIdx.x == 0) resolve_scales(p, s_enc);
+        __syncthreads();
+    }
+    TensorEncoder kenc, venc;
+    if (kWrite) {
+        kenc = s_enc[0];
+        venc = s_enc[1];
+    }
+
+    const bool small_slots = p.num_slots <= 0x7FFFFFFF;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint32_t kacc = 0, vacc = 0;
+
+    for (bool first = true; t < total; t += nwarps, first = false) {
+        if (!first) load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
+        const int64_t slot = r.slot;
         bool write_row = false;
         int64_t dst = 0;
         if (kWrite && slot >= 0) {
             if (slot >= p.num_slots) {
                 if (lane == 0) atomicOr(&g_error_word, kErrSlot);
-            } else {
+            } else if (!(kCross && t < p.num_tokens &&
+                         table_contains(s_table, log2, static_cast<uint32_t>(slot)))) {
                 int64_t blk, off;
                 if (p.block_shift >= 0) {
                     blk = slot >> p.block_shift;
@@ -358,48 +468,46 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
                 write_row = true;
             }
         }
+
         for (int c0 = 0; c0 < nchunks; c0 += 64) {
             const int ca = c0 + lane;
             const int cb = c0 + 32 + lane;
             const bool ha = ca < nchunks;
             const bool hb = cb < nchunks;
             if (c0 > 0) {   // rows wider than 512 elements: next 64 chunks
-                ka = ha ? ld_once(krow + ca * 8) : z;
-                kb = hb ? ld_once(krow + cb * 8) : z;
-                va = ha ? ld_once(vrow + ca * 8) : z;
-                vb = hb ? ld_once(vrow + cb * 8) : z;
+                r.ka = ha ? ld_once(r.k + ca * 8) : z;
+                r.kb = hb ? ld_once(r.k + cb * 8) : z;
+                r.va = ha ? ld_once(r.v + ca * 8) : z;
+                r.vb = hb ? ld_once(r.v + cb * 8) : z;
             }
             if (kAmax) {
-                kacc = absmax_uint4(absmax_uint4(kacc, ka), kb);
-                vacc = absmax_uint4(absmax_uint4(vacc, va), vb);
+                kacc = absmax_uint4(absmax_uint4(kacc, r.ka), r.kb);
+                vacc = absmax_uint4(absmax_uint4(vacc, r.va), r.vb);
             }
             if (kStage) {
                 const int64_t row = (p.stage_offset + t) * p.elems;
                 if (ha) {
-                    *reinterpret_cast<uint4 *>(p.stage_k + row + ca * 8) = ka;
-                    *reinterpret_cast<uint4 *>(p.stage_v + row + ca * 8) = va;
+                    *reinterpret_cast<uint4 *>(p.stage_k + row + ca * 8) = r.ka;
+                    *reinterpret_cast<uint4 *>(p.stage_v + row + ca * 8) = r.va;
                 }
                 if (hb) {
-                    *reinterpret_cast<uint4 *>(p.stage_k + row + cb * 8) = kb;
-                    *reinterpret_cast<uint4 *>(p.stage_v + row + cb * 8) = vb;
+                    *reinterpret_cast<uint4 *>(p.stage_k + row + cb * 8) = r.kb;
+                    *reinterpret_cast<uint4 *>(p.stage_v + row + cb * 8) = r.vb;
                 }
             }
             if (kWrite && write_row) {
-                if (sc.k.ok) {
-                    if (ha) *reinterpret_cast<uint2 *>(p.k_pool + dst + ca * 8) = sc.k.encode(ka);
-                    if (hb) *reinterpret_cast<uint2 *>(p.k_pool + dst + cb * 8) = sc.k.encode(kb);
+                if (kenc.ok) {
+                    if (ha) *reinterpret_cast<uint2 *>(p.k_pool + dst + ca * 8) = kenc.encode(r.ka);
+                    if (hb) *reinterpret_cast<uint2 *>(p.k_pool + dst + cb * 8) = kenc.encode(r.kb);
                 }
-                if (sc.v.ok) {
-                    if (ha) *reinterpret_cast<uint2 *>(p.v_pool + dst + ca * 8) = sc.v.encode(va);
-                    if (hb) *reinterpret_cast<uint2 *>(p.v_pool + dst + cb * 8) = sc.v.encode(vb);
+                if (venc.ok) {
+                    if (ha) *reinterpret_cast<uint2 *>(p.v_pool + dst + ca * 8) = venc.encode(r.va);
+                    if (hb) *reinterpret_cast<uint2 *>(p.v_pool + dst + cb * 8) = venc.encode(r.vb);
                 }
             }
         }
         if (kStage && lane == 0) p.stage_slots[p.stage_offset + t] = slot;
     }
-    // A freeze with nothing to rewrite still publishes the frozen scales.
-    if (kWrite && !scales_ready && p.freeze_amax != nullptr && blockIdx.x == 0)
-        sc.resolve(p);
 
     if (kAmax) {
         __shared__ uint32_t red[2][kKvWarps];
@@ -437,6 +545,12 @@ __global__ void calib_init_kernel(float *state) {
 // ---------------------------------------------------------------------------
 // launch geometry
 
+int table_log2_host(int64_t entries) {
+    int log2 = 6;
+    while ((int64_t{1} << log2) < 2 * entries) ++log2;
+    return log2;
+}
+
 struct DeviceInfo {
     int sms = 0;
 };
@@ -461,21 +575,27 @@ cudaError_t device_sms(int *sms) {
     return cudaSuccess;
 }
 
-// Resident CTAs per SM of a kernel, cached per (device, kernel).
+// Resident CTAs per SM of a kernel at a dynamic shared-memory size, cached
+// per (device, kernel, size).
 std::mutex g_occ_mutex;
-std::map<std::pair<int, const void *>, int> g_occ;
+std::map<std::tuple<int, const void *, size_t>, int> g_occ;
 
 template <typename Kernel>
-cudaError_t resident_ctas(Kernel kernel, int threads, int *out) {
+cudaError_t resident_ctas(Kernel kernel, int threads, size_t smem, int *out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kernel));
+    const auto key = std::make_tuple(dev, reinterpret_cast<const void *>(kernel), smem);
     std::lock_guard<std::mutex> lock(g_occ_mutex);
     auto it = g_occ.find(key);
     if (it == g_occ.end()) {
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem));
+            if (e != cudaSuccess) return e;
+        }
         int n = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
         if (e != cudaSuccess) return e;
         it = g_occ.emplace(key, n > 0 ? n : 1).first;
     }
@@ -484,11 +604,11 @@ cudaError_t resident_ctas(Kernel kernel, int threads, int *out) {
 }
 
 template <typename Kernel>
-cudaError_t grid_for(Kernel kernel, int threads, int64_t ctas_wanted, int *grid) {
+cudaError_t grid_for(Kernel kernel, int threads, size_t smem, int64_t ctas_wanted, int *grid) {
     int sms = 0, per_sm = 0;
     cudaError_t e = device_sms(&sms);
     if (e != cudaSuccess) return e;
-    e = resident_ctas(kernel, threads, &per_sm);
+    e = resident_ctas(kernel, threads, smem, &per_sm);
     if (e != cudaSuccess) return e;
     const int64_t cap = static_cast<int64_t>(sms) * per_sm;
     int64_t g = ctas_wanted < cap ? ctas_wanted : cap;
@@ -500,12 +620,12 @@ cudaError_t grid_for(Kernel kernel, int threads, int64_t ctas_wanted, int *grid)
 // Launch with programmatic stream serialization (see wait_for_previous_grid)
 // and count it.
 template <typename... Params, typename... Args>
-cudaError_t launch(void (*kernel)(Params...), int grid, int block, cudaStream_t stream,
-                   Args &&...args) {
+cudaError_t launch(void (*kernel)(Params...), int grid, int block, size_t smem,
+                   cudaStream_t stream, Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(static_cast<unsigned>(block));
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -518,14 +638,16 @@ cudaError_t launch(void (*kernel)(Params...), int grid, int block, cudaStream_t 
     return e;
 }
 
-template <bool A, bool S, bool W>
+template <bool A, bool S, bool W, bool X>
 cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
-    auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, 64> : kv_pass_kernel<A, S, W, 0>;
-    const int64_t wanted = (p.num_tokens + kKvWarps - 1) / kKvWarps;
+    auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, X, 64> : kv_pass_kernel<A, S, W, X, 0>;
+    const int64_t tokens = p.num_tokens + (X ? p.x_tokens : 0);
+    const int64_t wanted = (tokens + kKvWarps - 1) / kKvWarps;
+    const size_t smem = X ? (size_t{4} << table_log2_host(p.x_tokens)) : 0;
     int grid = 1;
-    cudaError_t e = grid_for(kernel, kKvThreads, wanted, &grid);
+    cudaError_t e = grid_for(kernel, kKvThreads, smem, wanted, &grid);
     if (e != cudaSuccess) return e;
-    return launch(kernel, grid, kKvThreads, stream, p);
+    return launch(kernel, grid, kKvThreads, smem, stream, p);
 }
 
 }  // namespace
@@ -540,25 +662,34 @@ cudaError_t launch_group_quant(const uint16_t *x, int64_t x_row_stride, uint8_t 
     int grid = 1;
     cudaError_t e;
     auto kernel = x_row_stride == k ? group_quant_kernel<true> : group_quant_kernel<false>;
-    e = grid_for(kernel, kGqThreads, wanted, &grid);
+    e = grid_for(kernel, kGqThreads, 0, wanted, &grid);
     if (e != cudaSuccess) return e;
-    return launch(kernel, grid, kGqThreads, stream, x, x_row_stride, q, scales, total,
+    return launch(kernel, grid, kGqThreads, 0, stream, x, x_row_stride, q, scales, total,
                   static_cast<uint32_t>(gpr));
+}
+
+bool can_merge_crossing(const KvPass &p) {
+    return p.x_tokens > 0 && p.x_tokens <= kMaxMergedCrossing && p.num_slots <= 0x7FFFFFFF;
 }
 
 cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
     const bool publish = p.do_write && p.freeze_amax != nullptr && p.scale_out != nullptr;
+    const bool cross = p.do_write && p.x_tokens > 0;
+    if (cross) {
+        if (!can_merge_crossing(p) || p.do_amax || p.do_stage) return cudaErrorInvalidValue;
+        return launch_kv_variant<false, false, true, true>(p, stream);
+    }
     if (p.num_tokens == 0 && !publish) return cudaSuccess;
-    if (p.do_amax && p.do_stage && p.do_write) return launch_kv_variant<true, true, true>(p, stream);
-    if (p.do_amax && p.do_stage) return launch_kv_variant<true, true, false>(p, stream);
-    if (p.do_amax && p.do_write) return launch_kv_variant<true, false, true>(p, stream);
-    if (p.do_amax) return launch_kv_variant<true, false, false>(p, stream);
-    if (p.do_write) return launch_kv_variant<false, false, true>(p, stream);
+    if (p.do_amax && p.do_stage && p.do_write) return launch_kv_variant<true, true, true, false>(p, stream);
+    if (p.do_amax && p.do_stage) return launch_kv_variant<true, true, false, false>(p, stream);
+    if (p.do_amax && p.do_write) return launch_kv_variant<true, false, true, false>(p, stream);
+    if (p.do_amax) return launch_kv_variant<true, false, false, false>(p, stream);
+    if (p.do_write) return launch_kv_variant<false, false, true, false>(p, stream);
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream) {
-    return launch(calib_init_kernel, 1, 1, stream, state_dev);
+    return launch(calib_init_kernel, 1, 1, 0, stream, state_dev);
 }
 
 int64_t launch_count() { return g_launch_count.load(std::memory_order_relaxed); }

@@ -76,10 +76,11 @@ def test_algorithmic_bytes():
     assert bench.GROUP_QUANT_BYTES == 71_283_360
     assert bench.PER_TOKEN["kv_write"] == 3080
     assert bench.PER_TOKEN["observe_stage_write"] == 5136
-    assert bench.launch_bytes("kv_write") == 498 * 3080
+    assert bench.launch_bytes("kv_write") == 4593 * 3080
+    assert bench.launch_bytes("replay_crossing") == (4095 + 498) * 3080
     assert bench.step_bytes(16) == 71_283_360 + 16 * (4095 * 5136 + 498 * 2048 + 4095 * 3080 +
                                                       498 * 3080)
-    assert len(bench.labels_of(16)) == 65
+    assert len(bench.labels_of(16)) == 49
 
 
 def test_cli_rejects_short_warmup():

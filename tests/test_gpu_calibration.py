@@ -114,6 +114,30 @@ def test_declined_batches(fused):
 
 
 @pytest.mark.parametrize("fused", [False, True])
+def test_crossing_batch_reuses_a_block_of_the_last_staged_batch(fused):
+    # batch 9 reaches the window and receives batch 8's second block: the
+    # replay of batch 8 and the crossing write touch the same 16 slots (one
+    # launch in the fused path), and the crossing tokens must end on top
+    spec, batches, _ = workloads.calib_window(recycle={6: (2, 1), 9: (8, 1)})
+    shared = set(batches[7].slot_mapping) & set(batches[8].slot_mapping)
+    assert len(shared) == 16
+    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused)
+    assert steps[8] == fp8q.STEP_FREEZE
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_crossing_batch_larger_than_one_merged_launch(fused):
+    # 9000 tokens reach a 1-token window at once: above the merge limit, the
+    # crossing batch gets a launch of its own after the scales are published
+    spec = workloads.large_kv_spec()
+    big = workloads.large_kv_layer(5, tokens=9000)
+    g, c, steps = _run_both(spec, [big], 1, 1.0, fused, check_every=True)
+    assert steps == [fp8q.STEP_FREEZE]
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
 def test_window_of_one_and_exact_window(fused):
     spec, batches, _ = workloads.calib_window(batch_sizes=(13, 32, 32))
     g, c, steps = _run_both(spec, batches, 1, 0.5, fused)

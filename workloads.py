@@ -185,16 +185,23 @@ CALIB_WINDOW = 256
 CALIB_BATCHES = (13,) + (32,) * 10   # 8 staged, batch 9 crosses, 2 after
 
 
-def calib_window(batch_sizes=CALIB_BATCHES, row_pad: int = 0):
-    """Calibration-window workload: returns (spec, batches, blocks per batch)."""
+def calib_window(batch_sizes=CALIB_BATCHES, row_pad: int = 0, recycle=None):
+    """Calibration-window workload: returns (spec, batches, blocks per batch).
+
+    ``recycle`` maps a batch number to (earlier batch number, block index):
+    before that batch, the earlier batch's block is freed and is the first
+    block the batch receives.  The default reuses batch 2's second block in
+    batch 6."""
+    recycle = {6: (2, 1)} if recycle is None else recycle
     spec = PoolSpec(128, 16, KV_HEADS, HEAD_DIM)
     g = generator(CALIB, 0, 0)
     alloc = BlockAllocator(spec.num_blocks, generator(CALIB, 0, 1))
     batches = []
     blocks_of = []
     for b, t in enumerate(batch_sizes, start=1):
-        if b == 6:
-            alloc.release(blocks_of[1][1])     # batch 2's second block
+        if b in recycle:
+            src, idx = recycle[b]
+            alloc.release(blocks_of[src - 1][idx])
         nblk = -(-t // spec.block_size)
         blocks = [alloc.alloc() for _ in range(nblk)]
         blocks_of.append(blocks)
