@@ -189,7 +189,7 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs, outputs, pools and calibrator state of one step."""
 
-    def __init__(self, device, layers: int) -> None:
+    def __init__(self, device, layers: int, flush: bool = True) -> None:
         import paged_kv_cache_group_b200 as fp8q
         self.fp8q = fp8q
         self.device = device
@@ -209,7 +209,7 @@ class Workload:
             self.v_pool.append(torch.full(shape, workloads.SENTINEL, dtype=torch.uint8, device=device))
         self.states = torch.zeros((layers, 4), dtype=torch.float32, device=device)
         self.states_init = torch.tensor([0.0, 0.0, 2.0, 2.0], device=device).repeat(layers, 1)
-        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size if flush else 16
         self.flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=device)
         self.flush_read = torch.ones(2 * l2, dtype=torch.uint8, device=device)
 
@@ -523,7 +523,21 @@ def measure_targets(w: Workload, stream, args) -> dict:
     out["kv_write_4593"] = {"us_per_layer": round(us, 3), "gbs": round(gbs, 1),
                             "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
                             "tokens_per_s": round(TOKENS / (us * 1e-6), 1),
-                            "bytes_per_layer": b}
+                            "bytes_per_layer": b,
+                            "launch": f"one launch per layer, {w.layers} back to back"}
+
+    def kvw_layers(mark):
+        fp8q.fp8_kv_write_layers(w.k, w.v, w.slots, w.k_pool, w.v_pool,
+                                 scale_devs=[scale] * w.layers)
+        mark(0)
+
+    us = timed(kvw_layers, 1)
+    gbs = b * w.layers / (us * 1e-6) / 1e9
+    out["kv_write_4593_all_layers"] = {"us": round(us, 3), "us_per_layer": round(us / w.layers, 3),
+                                       "gbs": round(gbs, 1),
+                                       "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                       "bytes": b * w.layers,
+                                       "launch": f"fp8_kv_write_layers: {w.layers} layers, one launch"}
     return out
 
 
@@ -586,6 +600,17 @@ def source_hash() -> str:
         with open(p, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+# ncu kernel of each bench label (the launch list names kernels, not labels)
+KERNEL_OF_LABEL = {
+    "group_quant": "group_quant_kernel<1>",
+    "observe_stage_write": "kv_pass_kernel<1, 1, 1, 0, 64>",
+    "amax": "kv_pass_kernel<1, 0, 0, 0, 64>",
+    "replay_crossing": "kv_pass_kernel<0, 0, 1, 1, 64>",
+    "kv_write": "kv_pass_kernel<0, 0, 1, 0, 64>",
+    "kv_write_layers": "kv_write_layers_kernel<64>",
+}
 
 
 def committed_traffic(label: str):
@@ -783,15 +808,25 @@ def run_calib(args) -> dict:
 
 
 def run_profile(args) -> None:
-    """A few eager steps on `--layers` layers, for an ncu capture of one kernel
-    (select it with ncu -k / -s / -c).  Prints nothing measured."""
+    """A few eager steps on `--layers` layers for an ncu capture: each step is
+    the bench step (group quant, then per layer the calibrating write) followed
+    by the steady-state write of every layer one launch each, then the same as
+    one fp8_kv_write_layers launch.  Select kernels with ncu -k / -s / -c.
+    ncu flushes caches itself, so no flush buffers are allocated."""
     torch.cuda.set_device(0)
-    w = Workload(torch.device("cuda", 0), args.layers)
+    dev = torch.device("cuda", 0)
+    w = Workload(dev, args.layers, flush=False)
+    scale = torch.tensor([0.05, 0.05], dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         for i in range(args.warmup + args.steps):
             w.reset(i)
             w.issue(w.calibrators())
+            for l in range(w.layers):
+                w.fp8q.fp8_kv_write(w.k[l], w.v[l], w.slots[l], w.k_pool[l], w.v_pool[l],
+                                    scale_dev=scale)
+            w.fp8q.fp8_kv_write_layers(w.k, w.v, w.slots, w.k_pool, w.v_pool,
+                                       scale_devs=[scale] * w.layers)
     torch.cuda.synchronize()
     assert w.fp8q.fp8q_device_error(clear=True) == 0
     print(json.dumps({"profile": "done", "layers": args.layers,

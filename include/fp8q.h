@@ -166,6 +166,46 @@ FP8Q_API fp8q_status fp8_kv_write(const void *k, const void *v,
                                   float v_scale, const float *scale_dev,
                                   void *stream);
 
+/* One layer's arguments of fp8_kv_write_layers. */
+typedef struct fp8q_kv_layer {
+    const void *k;                /* device bf16 rows, as for fp8_kv_write      */
+    const void *v;
+    const int64_t *slot_mapping;  /* device int64 [num_tokens]                  */
+    void *k_pool;                 /* this layer's pools                         */
+    void *v_pool;
+    const float *scale_dev;       /* device {k_scale, v_scale}, or NULL         */
+    float k_scale;                /* used when scale_dev is NULL                */
+    float v_scale;
+} fp8q_kv_layer;
+
+#define FP8Q_MAX_LAYERS 128
+
+/*
+ * fp8_kv_write_layers -- reshape_and_cache_fp8 for several layers in one launch.
+ *
+ * Source: as fp8_kv_write ("spark_model/layers/fp8_calibration/staging.rs",
+ * Fp8KvWriteTarget; "metrale_model_layers/layers/fp8_calibration.rs",
+ * module doc).  The pages write one layer per call; this performs exactly
+ * fp8_kv_write(layers[i], ...) for every i, as one grid (blockIdx.y = layer),
+ * for callers that hold all layers' K/V of a set of tokens at once (KV
+ * restored from host memory or a prefix cache, KV received from another
+ * device).  Layers are independent, so their order does not matter.
+ *
+ *   layers         HOST array [num_layers] of per-layer pointers and scales;
+ *                  alignment and scale rules as for fp8_kv_write
+ *   num_layers     0..FP8Q_MAX_LAYERS (0 is a no-op)
+ *   key_stride, value_stride, num_tokens, num_kv_heads, head_dim,
+ *   block_size, cache_stride, num_blocks
+ *                  shared by all layers, as for fp8_kv_write
+ * Returns FP8Q_OK, FP8Q_EINVAL, FP8Q_ECUDA.
+ */
+FP8Q_API fp8q_status fp8_kv_write_layers(const fp8q_kv_layer *layers,
+                                         int32_t num_layers, int64_t key_stride,
+                                         int64_t value_stride, int64_t num_tokens,
+                                         int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t block_size, int64_t cache_stride,
+                                         int64_t num_blocks, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* 3. Calibration                                                           */
 /* ------------------------------------------------------------------------ */

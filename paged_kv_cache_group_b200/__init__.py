@@ -119,6 +119,40 @@ def fp8_kv_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
         _stream(stream)))
 
 
+def fp8_kv_write_layers(ks, vs, slot_mappings, k_pools, v_pools, k_scales=None, v_scales=None,
+                        scale_devs=None, stream=None):
+    """reshape_and_cache_fp8 for several layers in one launch.  Per layer:
+    K, V ``[T, heads, dim]`` (same shape and row strides for all layers), an
+    int64 slot mapping and the layer's pools; scales by value (``k_scales``,
+    ``v_scales``) or from device ``scale_devs[i]``."""
+    n = len(ks)
+    if not (len(vs) == len(slot_mappings) == len(k_pools) == len(v_pools) == n):
+        raise ValueError("one k, v, slot_mapping, k_pool and v_pool per layer")
+    if n > _abi.MAX_LAYERS:
+        raise ValueError(f"at most {_abi.MAX_LAYERS} layers per launch")
+    if n == 0:
+        return
+    t, kst, e = _bf16_rows(ks[0], "k")
+    _, vst, _ = _bf16_rows(vs[0], "v")
+    heads, dim = ks[0].shape[1], ks[0].shape[2]
+    nb, bs, cs = _pool_geometry(k_pools[0], v_pools[0], e)
+    arr = (_abi.KvLayer * n)()
+    for i in range(n):
+        ti, ksi, _ = _bf16_rows(ks[i], "k")
+        _, vsi, _ = _bf16_rows(vs[i], "v")
+        if (ti, ksi, vsi) != (t, kst, vst) or tuple(ks[i].shape[1:]) != (heads, dim):
+            raise ValueError("all layers must share the row shape and strides")
+        if _pool_geometry(k_pools[i], v_pools[i], e) != (nb, bs, cs):
+            raise ValueError("all layers' pools must share one geometry")
+        sd = None if scale_devs is None else scale_devs[i]
+        arr[i] = _abi.KvLayer(_ptr(ks[i]), _ptr(vs[i]), _ptr(slot_mappings[i]), _ptr(k_pools[i]),
+                              _ptr(v_pools[i]), _ptr(sd),
+                              float(k_scales[i]) if k_scales is not None else 1.0,
+                              float(v_scales[i]) if v_scales is not None else 1.0)
+    _check("fp8_kv_write_layers", lib.fp8_kv_write_layers(
+        arr, n, kst, vst, t, heads, dim, bs, cs, nb, _stream(stream)))
+
+
 def fp8_kv_amax_observe(k: torch.Tensor, v: torch.Tensor, amax_dev: torch.Tensor, stream=None):
     """Max-accumulate max|K| and max|V| into the device fp32 ``amax_dev [2]``."""
     t, ks, e = _bf16_rows(k, "k")

@@ -37,11 +37,26 @@ class CalibStats(c.Structure):
     ]
 
 
+class KvLayer(c.Structure):
+    _fields_ = [
+        ("k", _P),
+        ("v", _P),
+        ("slot_mapping", _P),
+        ("k_pool", _P),
+        ("v_pool", _P),
+        ("scale_dev", _P),
+        ("k_scale", _F),
+        ("v_scale", _F),
+    ]
+
+
 SIGNATURES = {
     "fp8_group_quant": (STATUS, [_P, _I64, _P, _P, _I64, _I64, _P]),
     "fp8_kv_write": (STATUS, [_P, _P, _I64, _I64, _P, _I64, _I32, _I32, _P, _P, _I32, _I64,
                               _I64, _F, _F, _P, _P]),
     "fp8_kv_amax_observe": (STATUS, [_P, _P, _I64, _I64, _I64, _I32, _I32, _P, _P]),
+    "fp8_kv_write_layers": (STATUS, [c.POINTER(KvLayer), _I32, _I64, _I64, _I64, _I32, _I32,
+                                     _I32, _I64, _I64, _P]),
     "fp8_kv_calib_create": (STATUS, [_I64, _F, _I32, _I32, _P, _P, _P, _I64, _P, _P,
                                      c.POINTER(_P)]),
     "fp8_kv_calib_observe": (STATUS, [_P, _P, _P, _I64, _I64, _P, _I64, _I32, _I32, _P,
@@ -68,6 +83,7 @@ DEVERR_SLOT_OUT_OF_RANGE, DEVERR_BAD_SCALE = 0x1, 0x2
 MAX_STAGED_TOKENS = 4096
 PROVISIONAL_SCALE = 2.0
 CALIB_STATE_BYTES = 16
+MAX_LAYERS = 128
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 

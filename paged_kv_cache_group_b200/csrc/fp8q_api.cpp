@@ -306,6 +306,59 @@ FP8Q_API fp8q_status fp8_kv_write(const void *k, const void *v, int64_t key_stri
     return from_cuda(fp8q::launch_kv_pass(p, as_stream(stream)));
 }
 
+FP8Q_API fp8q_status fp8_kv_write_layers(const fp8q_kv_layer *layers, int32_t num_layers,
+                                         int64_t key_stride, int64_t value_stride,
+                                         int64_t num_tokens, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t block_size,
+                                         int64_t cache_stride, int64_t num_blocks, void *stream) {
+    if (num_layers < 0 || num_layers > FP8Q_MAX_LAYERS) return FP8Q_EINVAL;
+    if (num_layers > 0 && layers == nullptr) return FP8Q_EINVAL;
+    int64_t elems = 0;
+    // shapes are checked once; pointers per layer
+    if (!valid_rows(nullptr, nullptr, key_stride, value_stride, 0, num_kv_heads, head_dim, &elems))
+        return FP8Q_EINVAL;
+    if (num_tokens < 0) return FP8Q_EINVAL;
+    static_assert(FP8Q_MAX_LAYERS == fp8q::kMaxLayers, "layer limit");
+    fp8q::KvLayers L;
+    for (int32_t i = 0; i < num_layers; ++i) {
+        const fp8q_kv_layer &a = layers[i];
+        int64_t e = 0;
+        if (!valid_rows(a.k, a.v, key_stride, value_stride, num_tokens, num_kv_heads, head_dim, &e))
+            return FP8Q_EINVAL;
+        if (!valid_pools(a.k_pool, a.v_pool, block_size, cache_stride, num_blocks, elems))
+            return FP8Q_EINVAL;
+        if (num_tokens > 0 && (a.slot_mapping == nullptr || !aligned(a.slot_mapping, 8)))
+            return FP8Q_EINVAL;
+        if (a.scale_dev == nullptr) {
+            if (!(a.k_scale > 0.0f) || !(a.v_scale > 0.0f) || std::isinf(a.k_scale) ||
+                std::isinf(a.v_scale))
+                return FP8Q_EINVAL;
+        } else if (!aligned(a.scale_dev, 8)) {
+            return FP8Q_EINVAL;
+        }
+        fp8q::KvLayer &d = L.layer[i];
+        d.k = static_cast<const uint16_t *>(a.k);
+        d.v = static_cast<const uint16_t *>(a.v);
+        d.slot_mapping = a.slot_mapping;
+        d.k_pool = static_cast<uint8_t *>(a.k_pool);
+        d.v_pool = static_cast<uint8_t *>(a.v_pool);
+        d.scale_dev = a.scale_dev;
+        d.k_scale = a.k_scale;
+        d.v_scale = a.v_scale;
+    }
+    if (num_tokens == 0 || num_layers == 0) return FP8Q_OK;
+    L.key_stride = key_stride;
+    L.value_stride = value_stride;
+    L.num_tokens = num_tokens;
+    L.elems = static_cast<int32_t>(elems);
+    L.block_size = block_size;
+    L.block_shift = pow2_shift(block_size);
+    L.num_layers = num_layers;
+    L.cache_stride = cache_stride;
+    L.num_slots = num_blocks * block_size;
+    return from_cuda(fp8q::launch_kv_write_layers(L, as_stream(stream)));
+}
+
 FP8Q_API fp8q_status fp8_kv_amax_observe(const void *k, const void *v, int64_t key_stride,
                                          int64_t value_stride, int64_t num_tokens,
                                          int32_t num_kv_heads, int32_t head_dim, float *amax_dev,

@@ -68,6 +68,36 @@ struct KvPass {
     bool do_write = false;
 };
 
+// Several layers' writes in one launch (fp8_kv_write_layers): row strides,
+// shapes and pool geometry are shared, pointers and scales are per layer.
+constexpr int kMaxLayers = 128;
+
+struct KvLayer {
+    const uint16_t *k;
+    const uint16_t *v;
+    const int64_t *slot_mapping;
+    uint8_t *k_pool;
+    uint8_t *v_pool;
+    const float *scale_dev;   // {k_scale, v_scale} on the device, or null
+    float k_scale;
+    float v_scale;
+};
+
+struct KvLayers {
+    int64_t key_stride = 0;
+    int64_t value_stride = 0;
+    int64_t num_tokens = 0;
+    int32_t elems = 0;
+    int32_t block_size = 0;
+    int32_t block_shift = -1;
+    int32_t num_layers = 0;
+    int64_t cache_stride = 0;
+    int64_t num_slots = 0;
+    KvLayer layer[kMaxLayers];
+};
+
+cudaError_t launch_kv_write_layers(const KvLayers &p, cudaStream_t stream);
+
 cudaError_t launch_group_quant(const uint16_t *x, int64_t x_row_stride, uint8_t *q,
                                float *scales, int64_t m, int64_t k, cudaStream_t stream);
 

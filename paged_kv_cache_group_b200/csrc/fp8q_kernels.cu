@@ -189,17 +189,32 @@ struct TensorEncoder {
         lo2 = hi2 | 0x80008000u;
     }
 
-    __device__ __forceinline__ uint2 encode(uint4 w) const {
+    __device__ __forceinline__ static uint4 clamp4(uint4 w, uint32_t lo2, uint32_t hi2) {
+        w.x = clamp_bf16x2(w.x, lo2, hi2);
+        w.y = clamp_bf16x2(w.y, lo2, hi2);
+        w.z = clamp_bf16x2(w.z, lo2, hi2);
+        w.w = clamp_bf16x2(w.w, lo2, hi2);
+        return w;
+    }
+
+    // Two chunks of a row.  Only magnitudes at or beyond T can overflow
+    // x * r, and T is far above any realistic K/V, so the clamp runs only
+    // when the pair's largest magnitude reaches it.
+    __device__ __forceinline__ void encode2(uint4 a, uint4 b, uint2 &oa, uint2 &ob) const {
         if (fast) {
             if (clamp) {
-                w.x = clamp_bf16x2(w.x, lo2, hi2);
-                w.y = clamp_bf16x2(w.y, lo2, hi2);
-                w.z = clamp_bf16x2(w.z, lo2, hi2);
-                w.w = clamp_bf16x2(w.w, lo2, hi2);
+                const uint32_t m = absmax_bits16(absmax_uint4(absmax_uint4(0u, a), b));
+                if (m >= (hi2 & 0xFFFFu)) {
+                    a = clamp4(a, lo2, hi2);
+                    b = clamp4(b, lo2, hi2);
+                }
             }
-            return encode8(w, d);
+            oa = encode8(a, d);
+            ob = encode8(b, d);
+        } else {
+            oa = encode8_div(a, d.s);
+            ob = encode8_div(b, d.s);
         }
-        return encode8_div(w, d.s);
     }
 };
 
@@ -350,6 +365,15 @@ __device__ __forceinline__ void resolve_scales(const KvPass &p, TensorEncoder *e
     if (!(enc[0].ok && enc[1].ok) && blockIdx.x == 0) atomicOr(&g_error_word, kErrScale);
 }
 
+// Per-layer variant: a bad scale is reported by the first CTA of each layer.
+__device__ __forceinline__ void resolve_layer_scales(const KvPass &p, TensorEncoder *enc) {
+    const float ks = p.scale_dev != nullptr ? p.scale_dev[0] : p.k_scale;
+    const float vs = p.scale_dev != nullptr ? p.scale_dev[1] : p.v_scale;
+    enc[0].init(ks);
+    enc[1].init(vs);
+    if (!(enc[0].ok && enc[1].ok) && blockIdx.x == 0) atomicOr(&g_error_word, kErrScale);
+}
+
 // A token's row pointers (staged or crossing) and its first 64 chunks.
 struct Row {
     const uint16_t *k;
@@ -380,6 +404,99 @@ __device__ __forceinline__ void load_row(const KvPass &p, int64_t t, int lane, i
     r.vb = hb ? ld_once(r.v + (32 + lane) * 8) : z;
 }
 
+// One row of a pass: absmax, staging copy, and the quantized write into the
+// pool entry of its slot.
+template <bool kAmax, bool kStage, bool kWrite, bool kCross, int kChunks>
+__device__ __forceinline__ void process_row(const KvPass &p, Row &r, int64_t t, int lane,
+                                            int nchunks, const TensorEncoder &kenc,
+                                            const TensorEncoder &venc, const uint32_t *table,
+                                            int log2, bool small_slots, uint32_t &kacc,
+                                            uint32_t &vacc) {
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const int64_t slot = r.slot;
+    bool write_row = false;
+    int64_t dst = 0;
+    if (kWrite && slot >= 0) {
+        if (slot >= p.num_slots) {
+            if (lane == 0) atomicOr(&g_error_word, kErrSlot);
+        } else if (!(kCross && t < p.num_tokens &&
+                     table_contains(table, log2, static_cast<uint32_t>(slot)))) {
+            int64_t blk, off;
+            if (p.block_shift >= 0) {
+                blk = slot >> p.block_shift;
+                off = slot & ((int64_t{1} << p.block_shift) - 1);
+            } else if (small_slots) {
+                const uint32_t s32 = static_cast<uint32_t>(slot);
+                const uint32_t b32 = s32 / static_cast<uint32_t>(p.block_size);
+                blk = b32;
+                off = s32 - b32 * static_cast<uint32_t>(p.block_size);
+            } else {
+                blk = slot / p.block_size;
+                off = slot - blk * p.block_size;
+            }
+            dst = blk * p.cache_stride + off * p.elems;
+            write_row = true;
+        }
+    }
+
+    for (int c0 = 0; c0 < nchunks; c0 += 64) {
+        const int ca = c0 + lane;
+        const int cb = c0 + 32 + lane;
+        const bool ha = ca < nchunks;
+        const bool hb = cb < nchunks;
+        if (c0 > 0) {   // rows wider than 512 elements: next 64 chunks
+            r.ka = ha ? ld_once(r.k + ca * 8) : z;
+            r.kb = hb ? ld_once(r.k + cb * 8) : z;
+            r.va = ha ? ld_once(r.v + ca * 8) : z;
+            r.vb = hb ? ld_once(r.v + cb * 8) : z;
+        }
+        if (kAmax) {
+            kacc = absmax_uint4(absmax_uint4(kacc, r.ka), r.kb);
+            vacc = absmax_uint4(absmax_uint4(vacc, r.va), r.vb);
+        }
+        if (kStage) {
+            const int64_t row = (p.stage_offset + t) * p.elems;
+            if (ha) {
+                *reinterpret_cast<uint4 *>(p.stage_k + row + ca * 8) = r.ka;
+                *reinterpret_cast<uint4 *>(p.stage_v + row + ca * 8) = r.va;
+            }
+            if (hb) {
+                *reinterpret_cast<uint4 *>(p.stage_k + row + cb * 8) = r.kb;
+                *reinterpret_cast<uint4 *>(p.stage_v + row + cb * 8) = r.vb;
+            }
+        }
+        if (kWrite && write_row) {
+            uint2 oa, ob;
+            if (kenc.ok) {
+                kenc.encode2(r.ka, r.kb, oa, ob);
+                if (ha) *reinterpret_cast<uint2 *>(p.k_pool + dst + ca * 8) = oa;
+                if (hb) *reinterpret_cast<uint2 *>(p.k_pool + dst + cb * 8) = ob;
+            }
+            if (venc.ok) {
+                venc.encode2(r.va, r.vb, oa, ob);
+                if (ha) *reinterpret_cast<uint2 *>(p.v_pool + dst + ca * 8) = oa;
+                if (hb) *reinterpret_cast<uint2 *>(p.v_pool + dst + cb * 8) = ob;
+            }
+        }
+    }
+    if (kStage && lane == 0) p.stage_slots[p.stage_offset + t] = slot;
+}
+
+// Warm L2 with a token's K row (which 0), V row (1) or slot (2).
+template <bool kCross, bool kSlot>
+__device__ __forceinline__ void prefetch_row(const KvPass &p, int64_t t, int which) {
+    const bool crossing = kCross && t >= p.num_tokens;
+    const int64_t u = t - (crossing ? p.num_tokens : 0);
+    const uint32_t row_bytes = static_cast<uint32_t>(p.elems) * 2u;
+    if (which == 0)
+        prefetch_l2_bulk(crossing ? p.xk + u * p.x_key_stride : p.k + u * p.key_stride, row_bytes);
+    else if (which == 1)
+        prefetch_l2_bulk(crossing ? p.xv + u * p.x_value_stride : p.v + u * p.value_stride,
+                         row_bytes);
+    else if (kSlot)
+        prefetch_l2(crossing ? p.x_slots + u : p.slot_mapping + u);
+}
+
 // kChunks: 16-byte chunks per row when fixed at compile time (64 for the
 // common 4 x 128 rows), or 0 for any multiple of 8 elements.
 template <bool kAmax, bool kStage, bool kWrite, bool kCross, int kChunks>
@@ -395,18 +512,17 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     constexpr bool kSlot = kWrite || kStage;
 
     // the first token's K row, V row and slot into L2 while the previous
-    // kernel finishes
-    if (warp < total && lane < 3) {
-        const bool crossing = kCross && warp >= p.num_tokens;
-        const int64_t u = warp - (crossing ? p.num_tokens : 0);
-        const uint32_t row_bytes = static_cast<uint32_t>(p.elems) * 2u;
-        if (lane == 0)
-            prefetch_l2_bulk(crossing ? p.xk + u * p.x_key_stride : p.k + u * p.key_stride, row_bytes);
-        else if (lane == 1)
-            prefetch_l2_bulk(crossing ? p.xv + u * p.x_value_stride : p.v + u * p.value_stride,
-                             row_bytes);
-        else if (kSlot)
-            prefetch_l2(crossing ? p.x_slots + u : p.slot_mapping + u);
+    // kernel finishes (and, for a merged crossing batch, its slot list)
+    if (warp < total && lane < 3) prefetch_row<kCross, kSlot>(p, warp, lane);
+    // Only CTAs that rewrite staged tokens consult the crossing slots.  With
+    // the grid-stride loop a CTA's tokens are blockIdx.x*8 + k*nwarps + w, so
+    // a CTA whose first token is a crossing token never sees a staged one.
+    const bool need_table =
+        kCross && static_cast<int64_t>(blockIdx.x) * kKvWarps < p.num_tokens;
+    if (need_table && threadIdx.x == 32) {
+        const int64_t bytes = p.x_tokens * 8;
+        if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0)
+            prefetch_l2_bulk(p.x_slots, static_cast<uint32_t>(bytes));
     }
     wait_for_previous_grid();
     allow_next_grid();
@@ -418,9 +534,11 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
 
     // 2. per CTA: the crossing slots' hash set, and the scales
     int log2 = 0;
-    if (kCross) {
+    if (need_table) {
         log2 = table_log2(p.x_tokens);
-        for (int i = threadIdx.x; i < (1 << log2); i += kKvThreads) s_table[i] = kEmptySlot;
+        uint4 *tab4 = reinterpret_cast<uint4 *>(s_table);
+        const uint4 empty = make_uint4(kEmptySlot, kEmptySlot, kEmptySlot, kEmptySlot);
+        for (int i = threadIdx.x; i < (1 << log2) / 4; i += kKvThreads) tab4[i] = empty;
         __syncthreads();
         for (int64_t i = threadIdx.x; i < p.x_tokens; i += kKvThreads) {
             const int64_t s = __ldg(p.x_slots + i);
@@ -438,75 +556,13 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     }
 
     const bool small_slots = p.num_slots <= 0x7FFFFFFF;
-    const uint4 z = make_uint4(0, 0, 0, 0);
     uint32_t kacc = 0, vacc = 0;
 
     for (bool first = true; t < total; t += nwarps, first = false) {
         if (!first) load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
-        const int64_t slot = r.slot;
-        bool write_row = false;
-        int64_t dst = 0;
-        if (kWrite && slot >= 0) {
-            if (slot >= p.num_slots) {
-                if (lane == 0) atomicOr(&g_error_word, kErrSlot);
-            } else if (!(kCross && t < p.num_tokens &&
-                         table_contains(s_table, log2, static_cast<uint32_t>(slot)))) {
-                int64_t blk, off;
-                if (p.block_shift >= 0) {
-                    blk = slot >> p.block_shift;
-                    off = slot & ((int64_t{1} << p.block_shift) - 1);
-                } else if (small_slots) {
-                    const uint32_t s32 = static_cast<uint32_t>(slot);
-                    const uint32_t b32 = s32 / static_cast<uint32_t>(p.block_size);
-                    blk = b32;
-                    off = s32 - b32 * static_cast<uint32_t>(p.block_size);
-                } else {
-                    blk = slot / p.block_size;
-                    off = slot - blk * p.block_size;
-                }
-                dst = blk * p.cache_stride + off * p.elems;
-                write_row = true;
-            }
-        }
-
-        for (int c0 = 0; c0 < nchunks; c0 += 64) {
-            const int ca = c0 + lane;
-            const int cb = c0 + 32 + lane;
-            const bool ha = ca < nchunks;
-            const bool hb = cb < nchunks;
-            if (c0 > 0) {   // rows wider than 512 elements: next 64 chunks
-                r.ka = ha ? ld_once(r.k + ca * 8) : z;
-                r.kb = hb ? ld_once(r.k + cb * 8) : z;
-                r.va = ha ? ld_once(r.v + ca * 8) : z;
-                r.vb = hb ? ld_once(r.v + cb * 8) : z;
-            }
-            if (kAmax) {
-                kacc = absmax_uint4(absmax_uint4(kacc, r.ka), r.kb);
-                vacc = absmax_uint4(absmax_uint4(vacc, r.va), r.vb);
-            }
-            if (kStage) {
-                const int64_t row = (p.stage_offset + t) * p.elems;
-                if (ha) {
-                    *reinterpret_cast<uint4 *>(p.stage_k + row + ca * 8) = r.ka;
-                    *reinterpret_cast<uint4 *>(p.stage_v + row + ca * 8) = r.va;
-                }
-                if (hb) {
-                    *reinterpret_cast<uint4 *>(p.stage_k + row + cb * 8) = r.kb;
-                    *reinterpret_cast<uint4 *>(p.stage_v + row + cb * 8) = r.vb;
-                }
-            }
-            if (kWrite && write_row) {
-                if (kenc.ok) {
-                    if (ha) *reinterpret_cast<uint2 *>(p.k_pool + dst + ca * 8) = kenc.encode(r.ka);
-                    if (hb) *reinterpret_cast<uint2 *>(p.k_pool + dst + cb * 8) = kenc.encode(r.kb);
-                }
-                if (venc.ok) {
-                    if (ha) *reinterpret_cast<uint2 *>(p.v_pool + dst + ca * 8) = venc.encode(r.va);
-                    if (hb) *reinterpret_cast<uint2 *>(p.v_pool + dst + cb * 8) = venc.encode(r.vb);
-                }
-            }
-        }
-        if (kStage && lane == 0) p.stage_slots[p.stage_offset + t] = slot;
+        process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
+                                                            s_table, log2, small_slots, kacc,
+                                                            vacc);
     }
 
     if (kAmax) {
@@ -530,6 +586,54 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
             if (km) atomicMax(p.amax_bits + 0, km << 16);
             if (vm) atomicMax(p.amax_bits + 1, vm << 16);
         }
+    }
+}
+
+// Many layers' writes in one grid: blockIdx.y is the layer, blockIdx.x walks
+// that layer's tokens.  Per CTA, thread 0 resolves the layer's scales; the
+// rows go through the same code as a one-layer write.
+template <int kChunks>
+__global__ void __launch_bounds__(kKvThreads, 4) kv_write_layers_kernel(const KvLayers L) {
+    __shared__ TensorEncoder s_enc[2];
+    const KvLayer &ly = L.layer[blockIdx.y];
+    KvPass p;
+    p.k = ly.k;
+    p.v = ly.v;
+    p.key_stride = L.key_stride;
+    p.value_stride = L.value_stride;
+    p.slot_mapping = ly.slot_mapping;
+    p.num_tokens = L.num_tokens;
+    p.elems = L.elems;
+    p.k_pool = ly.k_pool;
+    p.v_pool = ly.v_pool;
+    p.block_size = L.block_size;
+    p.block_shift = L.block_shift;
+    p.cache_stride = L.cache_stride;
+    p.num_slots = L.num_slots;
+    p.scale_dev = ly.scale_dev;
+    p.k_scale = ly.k_scale;
+    p.v_scale = ly.v_scale;
+
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kKvThreads) >> 5;
+    const int nchunks = kChunks > 0 ? kChunks : (p.elems >> 3);
+    if (warp < p.num_tokens && lane < 3) prefetch_row<false, true>(p, warp, lane);
+    wait_for_previous_grid();
+    allow_next_grid();
+
+    Row r;
+    int64_t t = warp;
+    if (t < p.num_tokens) load_row<false, true, kChunks>(p, t, lane, nchunks, r);
+    if (threadIdx.x == 0) resolve_layer_scales(p, s_enc);
+    __syncthreads();
+    const TensorEncoder kenc = s_enc[0], venc = s_enc[1];
+    const bool small_slots = p.num_slots <= 0x7FFFFFFF;
+    uint32_t kacc = 0, vacc = 0;
+    for (bool first = true; t < p.num_tokens; t += nwarps, first = false) {
+        if (!first) load_row<false, true, kChunks>(p, t, lane, nchunks, r);
+        process_row<false, false, true, false, kChunks>(p, r, t, lane, nchunks, kenc, venc,
+                                                        nullptr, 0, small_slots, kacc, vacc);
     }
 }
 
@@ -686,6 +790,28 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
     if (p.do_amax) return launch_kv_variant<true, false, false, false>(p, stream);
     if (p.do_write) return launch_kv_variant<false, false, true, false>(p, stream);
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_kv_write_layers(const KvLayers &p, cudaStream_t stream) {
+    if (p.num_tokens == 0 || p.num_layers == 0) return cudaSuccess;
+    auto kernel = p.elems == 512 ? kv_write_layers_kernel<64> : kv_write_layers_kernel<0>;
+    const int64_t wanted = (p.num_tokens + kKvWarps - 1) / kKvWarps;
+    int gx = 1;
+    cudaError_t e = grid_for(kernel, kKvThreads, 0, wanted, &gx);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(p.num_layers));
+    cfg.blockDim = dim3(kKvThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e == cudaSuccess) g_launch_count.fetch_add(1, std::memory_order_relaxed);
+    return e;
 }
 
 cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream) {

@@ -197,3 +197,41 @@ def test_amax_matches_oracle_and_accumulates(case):
     fp8q.fp8_kv_amax_observe(_dev_rows(b.k, heads, dim), _dev_rows(b.v, heads, dim), amax2)
     got2 = host(amax2)
     assert got2[0] == np.float32(1e30) and got2[1] == want[1]
+
+
+def test_multi_layer_write_matches_the_oracle_per_layer():
+    """fp8_kv_write_layers = fp8_kv_write applied to each layer: four layers
+    with their own rows, slots (padding and an out-of-range slot in one), pools
+    and scales (by value, and from the device for one layer)."""
+    spec = workloads.large_kv_spec()
+    layers = [workloads.large_kv_layer(l, tokens=700) for l in (2, 3, 4, 5)]
+    layers[1].slot_mapping[::37] = -1
+    layers[2].slot_mapping[5] = spec.num_slots + 3
+    scales = [(0.05, 0.07), (2.0, 2.0), (600.0 / 448.0, 1e-30), (0.33, 0.44)]
+    n = spec.num_blocks * spec.cache_stride
+    kps = [torch.full((n,), workloads.SENTINEL, dtype=torch.uint8, device="cuda") for _ in layers]
+    vps = [torch.full((n,), workloads.SENTINEL, dtype=torch.uint8, device="cuda") for _ in layers]
+    shape = (spec.num_blocks, spec.block_size, spec.heads, spec.dim)
+    sd = torch.tensor(scales[3], dtype=torch.float32, device="cuda")
+    fp8q.fp8q_device_error(clear=True)
+    fp8q.fp8_kv_write_layers(
+        [_dev_rows(b.k, 4, 128) for b in layers], [_dev_rows(b.v, 4, 128) for b in layers],
+        [dev(b.slot_mapping) for b in layers], [p.view(shape) for p in kps],
+        [p.view(shape) for p in vps], k_scales=[s[0] for s in scales],
+        v_scales=[s[1] for s in scales], scale_devs=[None, None, None, sd])
+    err = fp8q.fp8q_device_error(clear=True)
+    assert err & fp8q.DEVERR_SLOT_OUT_OF_RANGE
+    for i, b in enumerate(layers):
+        ok, ov, _ = _oracle_write(spec, b, np.float32(scales[i][0]), np.float32(scales[i][1]))
+        assert np.array_equal(host(kps[i]), ok), f"layer {i} K: " + first_mismatch(host(kps[i]), ok)
+        assert np.array_equal(host(vps[i]), ov), f"layer {i} V: " + first_mismatch(host(vps[i]), ov)
+
+
+def test_multi_layer_write_zero_layers_and_tokens():
+    spec, b = workloads.tiny_kv()
+    fp8q.fp8_kv_write_layers([], [], [], [], [])
+    k = torch.empty((0, 4, 128), dtype=torch.bfloat16, device="cuda")
+    kp = _dev_pool(_pools(spec), spec)
+    fp8q.fp8_kv_write_layers([k], [k], [torch.empty(0, dtype=torch.int64, device="cuda")], [kp],
+                             [kp], k_scales=[1.0], v_scales=[1.0])
+    assert np.all(host(kp) == workloads.SENTINEL)
