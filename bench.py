@@ -511,6 +511,25 @@ def measure_targets(w: Workload, stream, args) -> dict:
                                          "launch": "mean of 4 back-to-back launches"}
     del xs, qs, ss
 
+    # the same activation for a GEMM padded to ceil16(M) rows: K-major scales
+    # and zeroed phantom rows in the same launch
+    m_pad = fp8q.ceil16(M)
+    qk = torch.empty((m_pad, K), dtype=torch.uint8, device=w.device)
+    sk = torch.empty((K // 128, m_pad), dtype=torch.float32, device=w.device)
+
+    def gqk(mark):
+        fp8q.fp8_group_quant_kmajor(w.x, m_pad, qk, sk)
+        mark(0)
+
+    usk = timed(gqk, 1)
+    bk = M * K * 2 + m_pad * K + m_pad * (K // 128) * 4
+    gbsk = bk / (usk * 1e-6) / 1e9
+    out["group_quant_kmajor_4593x5120"] = {"us": round(usk, 3), "gbs": round(gbsk, 1),
+                                           "frac_of_hbm": round(gbsk / peaks["hbm_gbs"], 4),
+                                           "m_pad": m_pad, "bytes": bk,
+                                           "launch": "single launch in its own graph"}
+    del qk, sk
+
     def kvw(mark):
         for l in range(w.layers):
             fp8q.fp8_kv_write(w.k[l], w.v[l], w.slots[l], w.k_pool[l], w.v_pool[l],
@@ -710,8 +729,10 @@ def run_reference(args) -> dict | None:
 def run_sweep(args) -> list[dict]:
     """Decode-width sweep: group quant at M in {1,2,4,8,16} x K in {5120,16384},
     1000 back-to-back launches per shape, timed as plain stream launches
-    through the binding and as a CUDA graph of 1000 launches.  Launch-bound by
-    design; inputs stay in L2, as they do in a decode loop."""
+    through the binding and as a CUDA graph of 1000 launches; once with the
+    row-major scales and once K-major with the phantom rows up to ceil16(M)
+    zeroed (the layout a padded FP8 GEMM reads).  Launch-bound by design;
+    inputs stay in L2, as they do in a decode loop."""
     import paged_kv_cache_group_b200 as fp8q
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
@@ -719,43 +740,52 @@ def run_sweep(args) -> list[dict]:
     n = 1000
     out = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for m in workloads.DECODE_MS:
-        for k in workloads.DECODE_KS:
-            bits = workloads.decode_quant(m, k)
-            x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
-            q = torch.empty((m, k), dtype=torch.uint8, device=dev)
-            sc = torch.empty((m, k // 128), dtype=torch.float32, device=dev)
-            with torch.cuda.stream(stream):
-                for _ in range(20):
-                    fp8q.fp8_group_quant(x, q, sc)
-                torch.cuda.synchronize()
-                plain = []
-                for _ in range(3):
-                    start.record()
+    for layout in ("row_major", "kmajor"):
+        for m in workloads.DECODE_MS:
+            for k in workloads.DECODE_KS:
+                bits = workloads.decode_quant(m, k)
+                x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+                rows = m if layout == "row_major" else fp8q.ceil16(m)
+                q = torch.empty((rows, k), dtype=torch.uint8, device=dev)
+                if layout == "row_major":
+                    sc = torch.empty((m, k // 128), dtype=torch.float32, device=dev)
+                    call = lambda: fp8q.fp8_group_quant(x, q, sc)             # noqa: E731
+                else:
+                    sc = torch.empty((k // 128, rows), dtype=torch.float32, device=dev)
+                    call = lambda: fp8q.fp8_group_quant_kmajor(x, rows, q, sc)  # noqa: E731
+                with torch.cuda.stream(stream):
+                    for _ in range(20):
+                        call()
+                    torch.cuda.synchronize()
+                    plain = []
+                    for _ in range(3):
+                        start.record()
+                        for _ in range(n):
+                            call()
+                        end.record()
+                        end.synchronize()
+                        plain.append(start.elapsed_time(end) * 1e3 / n)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
                     for _ in range(n):
-                        fp8q.fp8_group_quant(x, q, sc)
-                    end.record()
-                    end.synchronize()
-                    plain.append(start.elapsed_time(end) * 1e3 / n)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for _ in range(n):
-                    fp8q.fp8_group_quant(x, q, sc)
-            graph = []
-            with torch.cuda.stream(stream):
-                for _ in range(5):
-                    start.record()
-                    g.replay()
-                    end.record()
-                    end.synchronize()
-                    graph.append(start.elapsed_time(end) * 1e3 / n)
-            del g
-            b = m * k * 3 + m * (k // 128) * 4
-            us_p, us_g = statistics.median(plain), statistics.median(graph)
-            out.append({"m": m, "k": k, "bytes": b, "plain_us_per_launch": round(us_p, 3),
-                        "graph_us_per_launch": round(us_g, 3),
-                        "graph_gbs": round(b / (us_g * 1e-6) / 1e9, 1),
-                        "graph_tokens_per_s": round(m / (us_g * 1e-6), 1)})
+                        call()
+                graph = []
+                with torch.cuda.stream(stream):
+                    for _ in range(5):
+                        start.record()
+                        g.replay()
+                        end.record()
+                        end.synchronize()
+                        graph.append(start.elapsed_time(end) * 1e3 / n)
+                del g
+                # bytes read and written, phantom rows' zero codes and scales included
+                b = m * k * 2 + rows * k + rows * (k // 128) * 4
+                us_p, us_g = statistics.median(plain), statistics.median(graph)
+                out.append({"layout": layout, "m": m, "m_pad": rows, "k": k, "bytes": b,
+                            "plain_us_per_launch": round(us_p, 3),
+                            "graph_us_per_launch": round(us_g, 3),
+                            "graph_gbs": round(b / (us_g * 1e-6) / 1e9, 1),
+                            "graph_tokens_per_s": round(m / (us_g * 1e-6), 1)})
     return out
 
 

@@ -111,6 +111,42 @@ FP8Q_API fp8q_status fp8_group_quant(const void *x, int64_t x_row_stride,
                                      void *q, float *scales, int64_t m,
                                      int64_t k, void *stream);
 
+/*
+ * fp8_group_quant_kmajor -- the same quantization, laid out for a padded FP8
+ * GEMM: phantom rows zeroed and the scales transposed K-major, in one launch.
+ *
+ * Source: "spark_model/layers/ops/dispatch_proj_decode.rs",
+ * decode_w8a8_quant_act (quantize the rows, zero the codes of the phantom
+ * rows rows..ceil16(rows), re-lay the 1x128 scales out K-major over all m_pad
+ * rows, pad rows included), DecodeW8a8Plan (the cuBLASLt GEMM is handed
+ * m_pad = ceil16(M) rows) and the scale-layout clause of its doc (the GEMM
+ * reads the activation scales token-contiguous; the quantizer's [M, K/128]
+ * order gives wrong results on the same codes).  The pages do this as three
+ * launches (quantize, memset, transpose); here it is one pass.
+ *
+ * For r < m and g < k/128, with s and the codes exactly as fp8_group_quant:
+ *   q[r * k + 128g + j]       = E4M3(fp32(x[r, 128g + j] / s))
+ *   scales_km[g * m_pad + r]  = s
+ * and for m <= r < m_pad (phantom rows; x is not read):
+ *   q[r * k + 128g + j] = 0,  scales_km[g * m_pad + r] = 0.0f
+ *
+ *   x            device bf16, row r at x + r * x_row_stride; 16-byte aligned
+ *                (may be NULL when m == 0)
+ *   x_row_stride elements between rows; >= k, multiple of 8
+ *   q            device E4M3 [m_pad, k], packed rows; 8-byte aligned
+ *   scales_km    device fp32 [k/128, m_pad] (K-major); 4-byte aligned
+ *   m            live rows, >= 0
+ *   m_pad        rows of q and columns of scales_km, >= m (ceil16(m) for a
+ *                GEMM padded to 16 rows); 0 is a no-op
+ *   k            row width, a positive multiple of 128
+ * Returns FP8Q_OK, FP8Q_EINVAL (sizes, alignment, null pointers),
+ * FP8Q_ECUDA.
+ */
+FP8Q_API fp8q_status fp8_group_quant_kmajor(const void *x, int64_t x_row_stride,
+                                            void *q, float *scales_km,
+                                            int64_t m, int64_t m_pad, int64_t k,
+                                            void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* 2. Paged KV-cache quantize-and-scatter                                   */
 /* ------------------------------------------------------------------------ */
@@ -377,6 +413,24 @@ FP8Q_API fp8q_status fp8_kv_calib_observe_write(
     int32_t num_kv_heads, int32_t head_dim, void *k_pool, void *v_pool,
     int32_t block_size, int64_t cache_stride, int64_t num_blocks, void *stream,
     int32_t *step_out);
+
+/*
+ * fp8_kv_calib_restore -- start a calibrator frozen at saved scales.
+ *
+ * The pages keep the calibration state in memory only.  A server that
+ * restarts would otherwise calibrate every layer again (and keep CUDA graphs
+ * suppressed for the whole window).  A calibrator that has observed nothing
+ * yet can instead be frozen at scales saved earlier, e.g. read with
+ * fp8_kv_calib_read_state after a previous freeze: the call enqueues
+ * state_dev = {k_scale, v_scale, k_scale, v_scale} (the saved scales also
+ * stand in as the maxima) and every later observe is FP8Q_STEP_FROZEN.
+ *
+ *   k_scale, v_scale  finite and > 0
+ * Returns FP8Q_OK, FP8Q_EINVAL, FP8Q_ESTATE (the calibrator has already
+ * observed a batch), FP8Q_ECUDA.
+ */
+FP8Q_API fp8q_status fp8_kv_calib_restore(fp8_kv_calib *calib, float k_scale,
+                                          float v_scale, void *stream);
 
 /* Device pointer to {k_scale, v_scale} of the calibrator (state_dev + 2):
  * the provisional scale until the freeze, the frozen scales after it. */

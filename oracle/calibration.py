@@ -200,6 +200,22 @@ class Fp8KvCalibration:
     def scales(self):
         return (np.float32(self.state.k_scale), np.float32(self.state.v_scale))
 
+    def restore(self, k_scale, v_scale) -> None:
+        """Start frozen at scales saved from an earlier freeze.
+
+        Not on the pages (they keep the state in memory only); this is the
+        plainest extension of their state machine: a calibrator that has seen
+        no batch takes the frozen branch with the given scales, which also
+        stand in as the running maxima, and stages nothing."""
+        if self.state.frozen or self.state.tokens_seen != 0 or self.staging.used_tokens != 0:
+            raise RuntimeError("restore is only allowed before the first batch")
+        k_scale, v_scale = np.float32(k_scale), np.float32(v_scale)
+        if not (np.isfinite(k_scale) and np.isfinite(v_scale) and k_scale > 0 and v_scale > 0):
+            raise ValueError("saved scales must be finite and positive")
+        self.state.frozen = True
+        self.state.k_scale, self.state.v_scale = k_scale, v_scale
+        self.state.k_running_max, self.state.v_running_max = k_scale, v_scale
+
     def observe(self, k_bits, v_bits, num_tokens: int, num_kv_heads: int,
                 head_dim: int, target: Fp8KvWriteTarget) -> str:
         if not self.state.should_observe(num_tokens):

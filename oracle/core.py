@@ -114,6 +114,24 @@ def group_quant_strided(x_bits: np.ndarray, m: int, k: int, row_stride: int):
     return q, s
 
 
+def group_quant_kmajor(x_bits: np.ndarray, m: int, k: int, row_stride: int, m_pad: int):
+    """The activation quantized for a GEMM padded to ``m_pad`` rows, in the
+    steps of decode_w8a8_quant_act ("spark_model/layers/ops/
+    dispatch_proj_decode.rs"): quantize the m live rows; zero the codes of the
+    phantom rows m..m_pad-1; write every slot of the K-major scale array
+    ``[k/128, m_pad]``, the live rows' scales transposed and the pad rows 0.
+
+    Returns ``(codes uint8 [m_pad, k], scales_km float32 [k/128, m_pad])``."""
+    if m_pad < m:
+        raise ValueError("m_pad must be >= m")
+    q_live, s_live = group_quant_strided(x_bits, m, k, row_stride)
+    q = np.zeros((m_pad, k), dtype=np.uint8)          # phantom rows: zero codes
+    q[:m] = q_live
+    scales_km = np.zeros((k // GROUP, m_pad), dtype=np.float32)   # pad rows: zero scales
+    scales_km[:, :m] = s_live.T
+    return q, scales_km
+
+
 def absmax(x_bits: np.ndarray, rows: int, row_elems: int, row_stride: int) -> np.float32:
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     if rows > 0:

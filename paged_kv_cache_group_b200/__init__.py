@@ -79,6 +79,36 @@ def fp8_group_quant(x: torch.Tensor, q: torch.Tensor | None = None,
     return q, scales
 
 
+def ceil16(m: int) -> int:
+    """Rows a GEMM padded to 16-row tiles is handed for an m-row activation."""
+    return (m + 15) // 16 * 16
+
+
+def fp8_group_quant_kmajor(x: torch.Tensor, m_pad: int | None = None,
+                           q: torch.Tensor | None = None, scales_km: torch.Tensor | None = None,
+                           stream=None):
+    """Quantize a bf16 ``[m, k]`` activation for a padded FP8 GEMM: codes
+    ``q [m_pad, k]`` with rows m..m_pad-1 zero, and fp32 scales K-major
+    ``scales_km [k/128, m_pad]`` with the pad columns zero.  ``m_pad``
+    defaults to ceil16(m)."""
+    m, stride, k = _bf16_rows(x, "x")
+    m_pad = ceil16(m) if m_pad is None else int(m_pad)
+    if m_pad < m:
+        raise ValueError("m_pad must be >= the number of rows")
+    if q is None:
+        q = torch.empty((m_pad, k), dtype=torch.uint8, device=x.device)
+    if scales_km is None:
+        scales_km = torch.empty((k // 128, m_pad), dtype=torch.float32, device=x.device)
+    if q.dtype not in _BYTE_TYPES or not q.is_contiguous() or q.numel() < m_pad * k:
+        raise ValueError("q must be a contiguous uint8/float8_e4m3fn tensor of m_pad*k elements")
+    if scales_km.dtype != torch.float32 or not scales_km.is_contiguous() or \
+            scales_km.numel() < m_pad * (k // 128):
+        raise ValueError("scales_km must be a contiguous float32 tensor of (k/128)*m_pad elements")
+    _check("fp8_group_quant_kmajor", lib.fp8_group_quant_kmajor(
+        _ptr(x) if m else None, stride, _ptr(q), _ptr(scales_km), m, m_pad, k, _stream(stream)))
+    return q, scales_km
+
+
 # ---------------------------------------------------------------------------
 # paged KV write
 
@@ -252,6 +282,18 @@ class KvCalibration:
             ctypes.byref(step)))
         return step.value
 
+    def restore(self, k_scale: float, v_scale: float, stream=None) -> None:
+        """Start frozen at saved scales (only before the first observe)."""
+        _check("fp8_kv_calib_restore", lib.fp8_kv_calib_restore(
+            self.handle, float(k_scale), float(v_scale), _stream(stream)))
+
+    def saved_scales(self, stream=None) -> dict:
+        """The frozen scales as exact hex floats, for save_scales()/restore()."""
+        if self.stats()["state"] != 2:
+            raise Fp8qError("saved_scales", _abi.ESTATE, "the calibrator has not frozen")
+        _, _, ks, vs = self.read_state(stream)
+        return {"k_scale": float(ks).hex(), "v_scale": float(vs).hex()}
+
     def stats(self) -> dict:
         s = CalibStats()
         _check("fp8_kv_calib_stats_get", lib.fp8_kv_calib_stats_get(self.handle, ctypes.byref(s)))
@@ -286,6 +328,21 @@ def fp8_kv_calib_window_noalloc(k: torch.Tensor, v: torch.Tensor, slot_mapping: 
         _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), arr, len(counts), k.shape[1], k.shape[2],
         int(window_tokens), float(headroom), _ptr(k_pool), _ptr(v_pool), bs, cs, nb,
         _ptr(scales_out), _stream(stream)))
+
+
+def save_scales(calibrators, path: str) -> None:
+    """Write every layer's frozen scales to a JSON file (exact hex floats)."""
+    import json
+    with open(path, "w") as fh:
+        json.dump({"fp8_kv_scales": [c.saved_scales() for c in calibrators]}, fh, indent=1)
+
+
+def load_scales(path: str) -> list[tuple[float, float]]:
+    """Read scales written by save_scales(): [(k_scale, v_scale)] per layer."""
+    import json
+    with open(path) as fh:
+        data = json.load(fh)["fp8_kv_scales"]
+    return [(float.fromhex(d["k_scale"]), float.fromhex(d["v_scale"])) for d in data]
 
 
 def fp8q_device_error(clear: bool = True) -> int:

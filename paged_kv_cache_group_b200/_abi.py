@@ -52,6 +52,7 @@ class KvLayer(c.Structure):
 
 SIGNATURES = {
     "fp8_group_quant": (STATUS, [_P, _I64, _P, _P, _I64, _I64, _P]),
+    "fp8_group_quant_kmajor": (STATUS, [_P, _I64, _P, _P, _I64, _I64, _I64, _P]),
     "fp8_kv_write": (STATUS, [_P, _P, _I64, _I64, _P, _I64, _I32, _I32, _P, _P, _I32, _I64,
                               _I64, _F, _F, _P, _P]),
     "fp8_kv_amax_observe": (STATUS, [_P, _P, _I64, _I64, _I64, _I32, _I32, _P, _P]),
@@ -65,6 +66,7 @@ SIGNATURES = {
     "fp8_kv_calib_observe_write": (STATUS, [_P, _P, _P, _I64, _I64, _P, _I64, _I32, _I32, _P,
                                             _P, _I32, _I64, _I64, _P, c.POINTER(_I32)]),
     "fp8_kv_calib_scale_dev": (_P, [_P]),
+    "fp8_kv_calib_restore": (STATUS, [_P, _F, _F, _P]),
     "fp8_kv_calib_stats_get": (STATUS, [_P, c.POINTER(CalibStats)]),
     "fp8_kv_calib_read_state": (STATUS, [_P, _P, c.POINTER(_F)]),
     "fp8_kv_calib_destroy": (None, [_P]),

@@ -279,6 +279,20 @@ FP8Q_API fp8q_status fp8_group_quant(const void *x, int64_t x_row_stride, void *
                                               as_stream(stream)));
 }
 
+FP8Q_API fp8q_status fp8_group_quant_kmajor(const void *x, int64_t x_row_stride, void *q,
+                                            float *scales_km, int64_t m, int64_t m_pad,
+                                            int64_t k, void *stream) {
+    if (m < 0 || m_pad < m || k <= 0 || k % FP8Q_GROUP != 0) return FP8Q_EINVAL;
+    if (x_row_stride < k || x_row_stride % 8 != 0) return FP8Q_EINVAL;
+    if (m_pad == 0) return FP8Q_OK;
+    if (q == nullptr || scales_km == nullptr || (m > 0 && x == nullptr)) return FP8Q_EINVAL;
+    if (!aligned(x, 16) || !aligned(q, 8) || !aligned(scales_km, 4)) return FP8Q_EINVAL;
+    if (m_pad > INT64_MAX / x_row_stride || k / FP8Q_GROUP > 0xFFFFFFFF) return FP8Q_EINVAL;
+    return from_cuda(fp8q::launch_group_quant_kmajor(
+        static_cast<const uint16_t *>(x), x_row_stride, static_cast<uint8_t *>(q), scales_km, m,
+        m_pad, k, as_stream(stream)));
+}
+
 FP8Q_API fp8q_status fp8_kv_write(const void *k, const void *v, int64_t key_stride,
                                   int64_t value_stride, const int64_t *slot_mapping,
                                   int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
@@ -496,6 +510,22 @@ FP8Q_API fp8q_status fp8_kv_calib_observe_write(
     w.scale_dev = scale_dev(calib);
     return run_replay(calib, k_pool, v_pool, block_size, cache_stride, num_blocks, s, nullptr,
                       &w);
+}
+
+FP8Q_API fp8q_status fp8_kv_calib_restore(fp8_kv_calib *c, float k_scale, float v_scale,
+                                          void *stream) {
+    if (c == nullptr) return FP8Q_EINVAL;
+    if (!(k_scale > 0.0f) || !(v_scale > 0.0f) || std::isinf(k_scale) || std::isinf(v_scale))
+        return FP8Q_EINVAL;
+    if (c->phase != kCalibrating || c->tokens_seen != 0 || c->staged_batches != 0)
+        return FP8Q_ESTATE;
+    cudaError_t e = fp8q::launch_calib_set(c->state_dev, k_scale, v_scale, k_scale, v_scale,
+                                           as_stream(stream));
+    if (e != cudaSuccess) return FP8Q_ECUDA;
+    c->phase = kFrozen;
+    c->batches.clear();
+    c->used_tokens = 0;
+    return FP8Q_OK;
 }
 
 FP8Q_API const float *fp8_kv_calib_scale_dev(const fp8_kv_calib *calib) {

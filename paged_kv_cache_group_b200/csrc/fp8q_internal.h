@@ -110,8 +110,18 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream);
 constexpr int64_t kMaxMergedCrossing = 8192;
 bool can_merge_crossing(const KvPass &p);
 
+// Group quantization with phantom rows m..m_pad-1 zeroed and the scales
+// written K-major, scales_km[g * m_pad + r].
+cudaError_t launch_group_quant_kmajor(const uint16_t *x, int64_t x_row_stride, uint8_t *q,
+                                      float *scales_km, int64_t m, int64_t m_pad, int64_t k,
+                                      cudaStream_t stream);
+
 // Enqueues state_dev = {0, 0, 2.0, 2.0} (bit patterns of the fp32 values).
 cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream);
+
+// Enqueues state_dev = {a, b, c, d}.
+cudaError_t launch_calib_set(float *state_dev, float a, float b, float c, float d,
+                             cudaStream_t stream);
 
 // Number of kernels this library has launched in this process.
 int64_t launch_count();

@@ -235,6 +235,31 @@ __device__ __forceinline__ float freeze_scale(uint32_t amax_bits, float headroom
 
 constexpr int kGqThreads = 256;
 
+// One group of four lanes: load the 128 elements (zeros when !load), reduce
+// the group maximum and return the group's scale; the codes are left in c.
+__device__ __forceinline__ Divisor quant_group_load(const uint16_t *src, bool load, int ql,
+                                                   uint4 (&c)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        c[j] = load ? ld_once(src + (ql + 4 * j) * 8) : make_uint4(0, 0, 0, 0);
+
+    uint32_t acc = c[0].x;
+    acc = absmax_bf16x2(acc, c[0].y);
+    acc = absmax_bf16x2(acc, c[0].z);
+    acc = absmax_bf16x2(acc, c[0].w);
+#pragma unroll
+    for (int j = 1; j < 4; ++j) acc = absmax_uint4(acc, c[j]);
+    uint32_t m = absmax_bits16(acc);
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+
+    const float amax = __uint_as_float(m << 16);
+    Divisor d;
+    d.s = group_scale(fmaxf(amax, kScaleFloor));
+    d.r = __frcp_rn(d.s);
+    return d;
+}
+
 template <bool kPacked>
 __global__ void __launch_bounds__(kGqThreads)
 group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
@@ -260,33 +285,57 @@ group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
     for (int64_t o = warp; o < octets; o += nwarps) {
         const int64_t g = o * 8 + sub;
         const bool valid = g < total_groups;
-        const uint16_t *src = group_src(valid ? g : 0);
         uint4 c[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            c[j] = valid ? ld_once(src + (ql + 4 * j) * 8) : make_uint4(0, 0, 0, 0);
-
-        uint32_t acc = c[0].x;
-        acc = absmax_bf16x2(acc, c[0].y);
-        acc = absmax_bf16x2(acc, c[0].z);
-        acc = absmax_bf16x2(acc, c[0].w);
-#pragma unroll
-        for (int j = 1; j < 4; ++j) acc = absmax_uint4(acc, c[j]);
-        uint32_t m = absmax_bits16(acc);
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-
-        const float amax = __uint_as_float(m << 16);
-        Divisor d;
-        d.s = group_scale(fmaxf(amax, kScaleFloor));
-        d.r = __frcp_rn(d.s);
-
+        const Divisor d = quant_group_load(group_src(valid ? g : 0), valid, ql, c);
         if (valid) {
             uint8_t *dst = q + g * 128;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) = encode8(c[j], d);
             if (ql == 0) scales[g] = d.s;
+        }
+    }
+}
+
+// K-major variant.  A warp's eight groups are one column g of eight
+// consecutive rows, so their eight scales are adjacent in scales_km (one
+// 32-byte sector); consecutive warps take the next column of the same eight
+// rows, which keeps the grid's reads inside one slab of rows at a time.
+// Rows m..m_pad-1 are phantom: nothing is read, zeros are written.
+__global__ void __launch_bounds__(kGqThreads)
+group_quant_kmajor_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
+                          uint8_t *__restrict__ q, float *__restrict__ scales_km,
+                          int64_t m, int64_t m_pad, uint32_t groups_per_row) {
+    const int lane = threadIdx.x & 31;
+    const int sub = lane >> 2;
+    const int ql = lane & 3;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kGqThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGqThreads) >> 5;
+    const int64_t octets = ((m_pad + 7) >> 3) * groups_per_row;
+    const int64_t k = static_cast<int64_t>(groups_per_row) * 128;
+    if (lane < 8 && warp < octets) {
+        const int64_t ro = warp / groups_per_row;
+        const int64_t row = ro * 8 + lane;
+        if (row < m) prefetch_l2_bulk(x + row * x_row_stride + (warp - ro * groups_per_row) * 128, 256);
+    }
+    wait_for_previous_grid();
+    allow_next_grid();
+
+    for (int64_t o = warp; o < octets; o += nwarps) {
+        const int64_t ro = o / groups_per_row;
+        const int64_t col = o - ro * groups_per_row;
+        const int64_t row = ro * 8 + sub;
+        const bool live = row < m;
+        uint4 c[4];
+        const Divisor d =
+            quant_group_load(x + (live ? row * x_row_stride + col * 128 : 0), live, ql, c);
+        if (row < m_pad) {
+            uint8_t *dst = q + row * k + col * 128;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) =
+                    live ? encode8(c[j], d) : make_uint2(0, 0);
+            if (ql == 0) scales_km[col * m_pad + row] = live ? d.s : 0.0f;
         }
     }
 }
@@ -646,6 +695,15 @@ __global__ void calib_init_kernel(float *state) {
     state[3] = 2.0f;
 }
 
+__global__ void calib_set_kernel(float *state, float a, float b, float c, float d) {
+    wait_for_previous_grid();
+    allow_next_grid();
+    state[0] = a;
+    state[1] = b;
+    state[2] = c;
+    state[3] = d;
+}
+
 // ---------------------------------------------------------------------------
 // launch geometry
 
@@ -772,6 +830,20 @@ cudaError_t launch_group_quant(const uint16_t *x, int64_t x_row_stride, uint8_t 
                   static_cast<uint32_t>(gpr));
 }
 
+cudaError_t launch_group_quant_kmajor(const uint16_t *x, int64_t x_row_stride, uint8_t *q,
+                                      float *scales_km, int64_t m, int64_t m_pad, int64_t k,
+                                      cudaStream_t stream) {
+    const int64_t gpr = k / 128;
+    if (m_pad == 0) return cudaSuccess;
+    const int64_t warps = ((m_pad + 7) / 8) * gpr;
+    const int64_t wanted = (warps * 32 + kGqThreads - 1) / kGqThreads;
+    int grid = 1;
+    cudaError_t e = grid_for(group_quant_kmajor_kernel, kGqThreads, 0, wanted, &grid);
+    if (e != cudaSuccess) return e;
+    return launch(group_quant_kmajor_kernel, grid, kGqThreads, 0, stream, x, x_row_stride, q,
+                  scales_km, m, m_pad, static_cast<uint32_t>(gpr));
+}
+
 bool can_merge_crossing(const KvPass &p) {
     return p.x_tokens > 0 && p.x_tokens <= kMaxMergedCrossing && p.num_slots <= 0x7FFFFFFF;
 }
@@ -816,6 +888,11 @@ cudaError_t launch_kv_write_layers(const KvLayers &p, cudaStream_t stream) {
 
 cudaError_t launch_calib_init(float *state_dev, cudaStream_t stream) {
     return launch(calib_init_kernel, 1, 1, 0, stream, state_dev);
+}
+
+cudaError_t launch_calib_set(float *state_dev, float a, float b, float c, float d,
+                             cudaStream_t stream) {
+    return launch(calib_set_kernel, 1, 1, 0, stream, state_dev, a, b, c, d);
 }
 
 int64_t launch_count() { return g_launch_count.load(std::memory_order_relaxed); }

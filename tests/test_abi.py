@@ -107,6 +107,7 @@ def test_calibration_calls_reject_null_handles():
     assert L.fp8_kv_freeze_replay(None, None, None, 16, 8192, 1, None, None) == _abi.EINVAL
     assert L.fp8_kv_calib_stats_get(None, None) == _abi.EINVAL
     assert L.fp8_kv_calib_scale_dev(None) is None
+    assert L.fp8_kv_calib_restore(None, 1.0, 1.0, None) == _abi.EINVAL
     L.fp8_kv_calib_destroy(None)
 
 

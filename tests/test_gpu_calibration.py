@@ -234,3 +234,37 @@ def test_post_freeze_write_in_a_cuda_graph():
     assert np.array_equal(got[mask], eager[mask])
     assert np.all(got[~mask] == workloads.SENTINEL)
     del graph
+
+
+def test_saved_scales_restore_a_frozen_calibrator(tmp_path):
+    """Calibrate, save the frozen scales to a file, restore them into a fresh
+    calibrator (as after a restart) and write the whole window again: every
+    batch is FROZEN and the pools equal the oracle's restored calibrator."""
+    spec, batches, _ = workloads.calib_window()
+    g, c, _ = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, True, check_every=False)
+    path = str(tmp_path / "scales.json")
+    fp8q.save_scales([g.cal], path)
+    (ks, vs), = fp8q.load_scales(path)
+    assert (np.float32(ks), np.float32(vs)) == c.scales()
+
+    fresh = GpuLayer(spec, workloads.CALIB_WINDOW, 1.0, fused=True)
+    fresh.cal.restore(ks, vs)
+    oc, kp, vp = _oracle_layer(spec, workloads.CALIB_WINDOW, 1.0)
+    oc.restore(ks, vs)
+    assert fresh.cal.stats()["state"] == 2
+    assert [fresh.step(b) for b in batches] == [fp8q.STEP_FROZEN] * len(batches)
+    cal.run_calibrated_writes(oc, [cal.KvBatch(b.k, b.v, b.slot_mapping, b.key_stride,
+                                               b.value_stride) for b in batches],
+                              spec.heads, spec.dim, kp, vp, spec.block_size, spec.cache_stride,
+                              spec.num_blocks)
+    gk, gv = host(fresh.kp), host(fresh.vp)
+    assert np.array_equal(gk, kp), first_mismatch(gk, kp)
+    assert np.array_equal(gv, vp), first_mismatch(gv, vp)
+    ka, va, rks, rvs = fresh.cal.read_state()
+    assert (np.float32(ka), np.float32(va)) == (oc.state.k_running_max, oc.state.v_running_max)
+    assert (np.float32(rks), np.float32(rvs)) == oc.scales()
+    # restoring is only allowed before the first observe
+    with pytest.raises(fp8q.Fp8qError) as ei:
+        g.cal.restore(ks, vs)
+    assert ei.value.status == -3
+    fresh.cal.close()

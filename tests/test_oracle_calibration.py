@@ -197,3 +197,32 @@ def test_graph_readiness():
     assert not cal.graphs_ready_after_fp8_kv_cal([True, False, None])
     assert cal.dtype_runs_online_fp8_kv_calibration("fp8")
     assert not cal.dtype_runs_online_fp8_kv_calibration("bf16")
+
+
+def test_restored_calibrator_writes_like_brute_force_at_the_saved_scales():
+    """A calibrator restored at saved scales is frozen from its first batch:
+    every batch is written once, in order, at those scales (brute force), no
+    batch is staged and the maxima read back as the scales."""
+    spec, batches, _ = workloads.calib_window()
+    done, _, _, _ = _run_window(workloads.CALIB_WINDOW, 1.0, batches, spec)
+    saved = done.scales()
+    c = cal.Fp8KvCalibration(0, workloads.CALIB_WINDOW, 1.0)
+    c.restore(*saved)
+    kp, vp = spec.new_pool().reshape(-1), spec.new_pool().reshape(-1)
+    run = cal.run_calibrated_writes(c, _as_oracle_batches(batches), spec.heads, spec.dim,
+                                    kp, vp, spec.block_size, spec.cache_stride, spec.num_blocks)
+    assert run.steps == [cal.FROZEN] * len(batches)
+    ek, ev = _bruteforce_pools(spec, batches, [(i, saved) for i in range(len(batches))])
+    assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
+    assert c.staging.used_tokens == 0 and c.freeze_log is None
+    assert (c.state.k_running_max, c.state.v_running_max) == saved
+
+
+def test_restore_rejects_late_calls_and_bad_scales():
+    spec, batches, _ = workloads.calib_window()
+    c, _, _, _ = _run_window(workloads.CALIB_WINDOW, 1.0, batches[:1], spec)
+    with pytest.raises(RuntimeError):
+        c.restore(1.0, 1.0)
+    for bad in ((0.0, 1.0), (1.0, -2.0), (float("inf"), 1.0), (1.0, float("nan"))):
+        with pytest.raises(ValueError):
+            cal.Fp8KvCalibration(0, 8, 1.0).restore(*bad)
