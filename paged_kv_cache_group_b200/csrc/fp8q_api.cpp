@@ -163,7 +163,7 @@ fp8q_status plan_observe(fp8_kv_calib *c, const void *k, const void *v, int64_t 
 // replay.  Either way each slot ends with its last writer in arrival order.
 fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t block_size,
                        int64_t cache_stride, int64_t num_blocks, cudaStream_t stream,
-                       int64_t *replayed, const KvPass *crossing) {
+                       int64_t *replayed, const KvPass *crossing, bool chained = false) {
     if (c->phase != kFreezePending) return FP8Q_ESTATE;
     if (!valid_pools(k_pool, v_pool, block_size, cache_stride, num_blocks, c->elems))
         return FP8Q_EINVAL;
@@ -181,6 +181,10 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
     p.freeze_amax = amax_bits(c);
     p.headroom = c->headroom;
     p.scale_out = scale_dev(c);
+    // chained: the previous launch on the stream is this call's own amax pass,
+    // and every launch below follows one of these; the staged rows and the
+    // crossing batch were all written before that amax pass was enqueued.
+    p.early_loads = chained;
 
     // Last staged batch with rows: the one the crossing batch joins.
     int64_t last = -1;
@@ -228,7 +232,9 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
             if (fp8q::launch_kv_pass(p, stream) != cudaSuccess) return FP8Q_ECUDA;
         }
         if (crossing != nullptr && !merge) {
-            if (fp8q::launch_kv_pass(*crossing, stream) != cudaSuccess) return FP8Q_ECUDA;
+            KvPass q = *crossing;
+            q.early_loads = chained;
+            if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
         }
     }
     const int64_t batches = static_cast<int64_t>(c->batches.size());
@@ -508,8 +514,9 @@ FP8Q_API fp8q_status fp8_kv_calib_observe_write(
     cudaError_t e = fp8q::launch_kv_pass(p, s);
     if (e != cudaSuccess) return FP8Q_ECUDA;
     w.scale_dev = scale_dev(calib);
+    // the amax pass above is enqueued only when the batch has tokens
     return run_replay(calib, k_pool, v_pool, block_size, cache_stride, num_blocks, s, nullptr,
-                      &w);
+                      &w, /*chained=*/p.num_tokens > 0);
 }
 
 FP8Q_API fp8q_status fp8_kv_calib_restore(fp8_kv_calib *c, float k_scale, float v_scale,

@@ -66,6 +66,15 @@ struct KvPass {
     bool do_amax = false;
     bool do_stage = false;
     bool do_write = false;
+    // The launch directly before this one on the stream is a kernel of this
+    // library, and nothing this pass reads (rows, slots, crossing slots) is
+    // written by it.  Every kernel here passes its dependency wait before it
+    // lets its dependents start, so everything enqueued before that kernel has
+    // completed by the time this pass starts: the pass may then load its rows
+    // and build its crossing-slot table before its own wait.  Only scales
+    // produced by the previous kernel and the stores wait.  Set only where a
+    // call enqueues that whole chain itself.
+    bool early_loads = false;
 };
 
 // Several layers' writes in one launch (fp8_kv_write_layers): row strides,

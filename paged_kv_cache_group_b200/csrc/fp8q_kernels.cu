@@ -41,7 +41,6 @@ __device__ uint32_t g_error_word;
 
 namespace {
 
-constexpr float kE4m3Max = 448.0f;
 constexpr float kScaleFloor = 1e-12f;
 constexpr uint32_t kErrSlot = 0x1u;
 constexpr uint32_t kErrScale = 0x2u;
@@ -80,9 +79,6 @@ __device__ __forceinline__ void allow_next_grid() {
 // a later load still returns whatever the previous kernel wrote.
 __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
 }
 
 // Per-half max of |a| and |b| for two bf16x2 words (the sign bits of the
@@ -219,9 +215,11 @@ struct TensorEncoder {
 };
 
 // Frozen scale: max(amax * headroom, 1e-12) / 448, product rounded first.
+// The division is group_scale's exact RN(y / 448) (y is a normal fp32 here);
+// an infinite product stays infinite, as in IEEE division.
 __device__ __forceinline__ float freeze_scale(uint32_t amax_bits, float headroom) {
-    const float widened = __fmul_rn(__uint_as_float(amax_bits), headroom);
-    return __fdiv_rn(fmaxf(widened, kScaleFloor), kE4m3Max);
+    const float y = fmaxf(__fmul_rn(__uint_as_float(amax_bits), headroom), kScaleFloor);
+    return y < INFINITY ? group_scale(y) : y;
 }
 
 // ---------------------------------------------------------------------------
@@ -386,41 +384,75 @@ __device__ __forceinline__ bool table_contains(const uint32_t *tab, int log2, ui
     return false;
 }
 
-__device__ __forceinline__ int table_log2(int64_t entries) {
+// Pools of at most this many slots take an exact bitmap of the crossing slots
+// (one bit per slot, 32 KB of shared memory at most) instead of the hash set.
+constexpr int64_t kBitmapMaxSlots = int64_t{1} << 18;
+
+// Hash-set size for `entries` crossing slots: load factor at most 1/4 up to
+// 4096 entries, at most 1/2 above (64 KB at the 8192-slot merge limit).
+__host__ __device__ __forceinline__ int table_log2(int64_t entries) {
+    const int64_t want = entries <= 4096 ? 4 * entries : 2 * entries;
     int log2 = 6;
-    while ((int64_t{1} << log2) < 2 * entries) ++log2;
+    while ((int64_t{1} << log2) < want) ++log2;
     return log2;
 }
 
-// Scales of a write pass (see KvPass), resolved by one thread.
-__device__ __forceinline__ void resolve_scales(const KvPass &p, TensorEncoder *enc) {
+// Shared-memory bytes of the crossing set of a merged launch.
+__host__ __device__ __forceinline__ int64_t crossing_set_bytes(int64_t num_slots,
+                                                              int64_t x_tokens) {
+    if (num_slots <= kBitmapMaxSlots) return ((num_slots + 127) >> 7) * 16;
+    return int64_t{4} << table_log2(x_tokens);
+}
+
+// Membership in the crossing set: log2 == 0 is the slot bitmap.
+__device__ __forceinline__ bool crossing_contains(const uint32_t *tab, int log2, uint32_t key) {
+    if (log2 == 0) return (tab[key >> 5] >> (key & 31u)) & 1u;
+    return table_contains(tab, log2, key);
+}
+
+// Scales of a write pass (see KvPass).  Every warp resolves them itself from
+// two loads issued together with its row loads; a CTA-wide broadcast through
+// shared memory would put a barrier behind the slowest of those loads.  Lane 0
+// of the grid's first warp reports a bad scale and, for a freeze, publishes
+// the frozen scales.
+__device__ __forceinline__ void resolve_scales(const KvPass &p, TensorEncoder &kenc,
+                                               TensorEncoder &venc) {
     float ks, vs;
     if (p.freeze_amax != nullptr) {
-        ks = freeze_scale(p.freeze_amax[0], p.headroom);
-        vs = freeze_scale(p.freeze_amax[1], p.headroom);
-        if (p.scale_out != nullptr && blockIdx.x == 0) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(p.freeze_amax);
+        ks = freeze_scale(a.x, p.headroom);
+        vs = freeze_scale(a.y, p.headroom);
+        if (p.scale_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
             p.scale_out[0] = ks;
             p.scale_out[1] = vs;
         }
     } else if (p.scale_dev != nullptr) {
-        ks = p.scale_dev[0];
-        vs = p.scale_dev[1];
+        const float2 sd = *reinterpret_cast<const float2 *>(p.scale_dev);
+        ks = sd.x;
+        vs = sd.y;
     } else {
         ks = p.k_scale;
         vs = p.v_scale;
     }
-    enc[0].init(ks);
-    enc[1].init(vs);
-    if (!(enc[0].ok && enc[1].ok) && blockIdx.x == 0) atomicOr(&g_error_word, kErrScale);
+    kenc.init(ks);
+    venc.init(vs);
+    if (!(kenc.ok && venc.ok) && blockIdx.x == 0 && threadIdx.x == 0)
+        atomicOr(&g_error_word, kErrScale);
 }
 
 // Per-layer variant: a bad scale is reported by the first CTA of each layer.
-__device__ __forceinline__ void resolve_layer_scales(const KvPass &p, TensorEncoder *enc) {
-    const float ks = p.scale_dev != nullptr ? p.scale_dev[0] : p.k_scale;
-    const float vs = p.scale_dev != nullptr ? p.scale_dev[1] : p.v_scale;
-    enc[0].init(ks);
-    enc[1].init(vs);
-    if (!(enc[0].ok && enc[1].ok) && blockIdx.x == 0) atomicOr(&g_error_word, kErrScale);
+__device__ __forceinline__ void resolve_layer_scales(const KvPass &p, TensorEncoder &kenc,
+                                                     TensorEncoder &venc) {
+    float ks = p.k_scale, vs = p.v_scale;
+    if (p.scale_dev != nullptr) {
+        const float2 sd = *reinterpret_cast<const float2 *>(p.scale_dev);
+        ks = sd.x;
+        vs = sd.y;
+    }
+    kenc.init(ks);
+    venc.init(vs);
+    if (!(kenc.ok && venc.ok) && blockIdx.x == 0 && threadIdx.x == 0)
+        atomicOr(&g_error_word, kErrScale);
 }
 
 // A token's row pointers (staged or crossing) and its first 64 chunks.
@@ -469,7 +501,7 @@ __device__ __forceinline__ void process_row(const KvPass &p, Row &r, int64_t t, 
         if (slot >= p.num_slots) {
             if (lane == 0) atomicOr(&g_error_word, kErrSlot);
         } else if (!(kCross && t < p.num_tokens &&
-                     table_contains(table, log2, static_cast<uint32_t>(slot)))) {
+                     crossing_contains(table, log2, static_cast<uint32_t>(slot)))) {
             int64_t blk, off;
             if (p.block_shift >= 0) {
                 blk = slot >> p.block_shift;
@@ -531,19 +563,19 @@ __device__ __forceinline__ void process_row(const KvPass &p, Row &r, int64_t t, 
     if (kStage && lane == 0) p.stage_slots[p.stage_offset + t] = slot;
 }
 
-// Warm L2 with a token's K row (which 0), V row (1) or slot (2).
-template <bool kCross, bool kSlot>
-__device__ __forceinline__ void prefetch_row(const KvPass &p, int64_t t, int which) {
+// Warm L2 with the K row (lane 0) or the V row (lane 1) of token t; pointers
+// are chosen by selects, so the two lanes do not diverge.
+template <bool kCross>
+__device__ __forceinline__ void prefetch_row(const KvPass &p, int64_t t, int lane) {
     const bool crossing = kCross && t >= p.num_tokens;
-    const int64_t u = t - (crossing ? p.num_tokens : 0);
-    const uint32_t row_bytes = static_cast<uint32_t>(p.elems) * 2u;
-    if (which == 0)
-        prefetch_l2_bulk(crossing ? p.xk + u * p.x_key_stride : p.k + u * p.key_stride, row_bytes);
-    else if (which == 1)
-        prefetch_l2_bulk(crossing ? p.xv + u * p.x_value_stride : p.v + u * p.value_stride,
-                         row_bytes);
-    else if (kSlot)
-        prefetch_l2(crossing ? p.x_slots + u : p.slot_mapping + u);
+    const int64_t u = crossing ? t - p.num_tokens : t;
+    const uint16_t *base = lane ? p.v : p.k;
+    int64_t stride = lane ? p.value_stride : p.key_stride;
+    if (kCross && crossing) {
+        base = lane ? p.xv : p.xk;
+        stride = lane ? p.x_value_stride : p.x_key_stride;
+    }
+    prefetch_l2_bulk(base + u * stride, static_cast<uint32_t>(p.elems) * 2u);
 }
 
 // kChunks: 16-byte chunks per row when fixed at compile time (64 for the
@@ -551,7 +583,6 @@ __device__ __forceinline__ void prefetch_row(const KvPass &p, int64_t t, int whi
 template <bool kAmax, bool kStage, bool kWrite, bool kCross, int kChunks>
 __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) {
     extern __shared__ uint32_t s_table[];        // crossing slots (kCross)
-    __shared__ TensorEncoder s_enc[2];
 
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
@@ -560,55 +591,73 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     const int64_t total = p.num_tokens + (kCross ? p.x_tokens : 0);
     constexpr bool kSlot = kWrite || kStage;
 
-    // the first token's K row, V row and slot into L2 while the previous
-    // kernel finishes (and, for a merged crossing batch, its slot list)
-    if (warp < total && lane < 3) prefetch_row<kCross, kSlot>(p, warp, lane);
     // Only CTAs that rewrite staged tokens consult the crossing slots.  With
     // the grid-stride loop a CTA's tokens are blockIdx.x*8 + k*nwarps + w, so
     // a CTA whose first token is a crossing token never sees a staged one.
     const bool need_table =
         kCross && static_cast<int64_t>(blockIdx.x) * kKvWarps < p.num_tokens;
-    if (need_table && threadIdx.x == 32) {
-        const int64_t bytes = p.x_tokens * 8;
-        if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0)
-            prefetch_l2_bulk(p.x_slots, static_cast<uint32_t>(bytes));
+    const bool early = p.early_loads;
+    if (!early) {
+        // the first token's K row, V row and slot into L2 while the previous
+        // kernel finishes (and, for a merged crossing batch, its slot list)
+        if (warp < total && lane < 2) prefetch_row<kCross>(p, warp, lane);
+        if (need_table && threadIdx.x == 32) {
+            const int64_t bytes = p.x_tokens * 8;
+            if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0)
+                prefetch_l2_bulk(p.x_slots, static_cast<uint32_t>(bytes));
+        }
+        wait_for_previous_grid();
+        allow_next_grid();
     }
-    wait_for_previous_grid();
-    allow_next_grid();
 
     // 1. this warp's first token: loads out first
     Row r;
     int64_t t = warp;
     if (t < total) load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
 
-    // 2. per CTA: the crossing slots' hash set, and the scales
+    // 2. per CTA: the crossing slots, as a bitmap over the pool's slots or,
+    // for larger pools, a hash set
     int log2 = 0;
     if (need_table) {
-        log2 = table_log2(p.x_tokens);
+        const bool bitmap = p.num_slots <= kBitmapMaxSlots;
+        log2 = bitmap ? 0 : table_log2(p.x_tokens);
         uint4 *tab4 = reinterpret_cast<uint4 *>(s_table);
-        const uint4 empty = make_uint4(kEmptySlot, kEmptySlot, kEmptySlot, kEmptySlot);
-        for (int i = threadIdx.x; i < (1 << log2) / 4; i += kKvThreads) tab4[i] = empty;
+        const int n4 = static_cast<int>(crossing_set_bytes(p.num_slots, p.x_tokens) >> 4);
+        const uint32_t f = bitmap ? 0u : kEmptySlot;
+        const uint4 fill = make_uint4(f, f, f, f);
+        for (int i = threadIdx.x; i < n4; i += kKvThreads) tab4[i] = fill;
         __syncthreads();
         for (int64_t i = threadIdx.x; i < p.x_tokens; i += kKvThreads) {
-            const int64_t s = __ldg(p.x_slots + i);
-            if (s >= 0 && s < p.num_slots) table_insert(s_table, log2, static_cast<uint32_t>(s));
+            const int64_t sl = __ldg(p.x_slots + i);
+            if (sl >= 0 && sl < p.num_slots) {
+                const uint32_t key = static_cast<uint32_t>(sl);
+                if (bitmap)
+                    atomicOr(&s_table[key >> 5], 1u << (key & 31u));
+                else
+                    table_insert(s_table, log2, key);
+            }
         }
-    }
-    if (kWrite) {
-        if (threadIdx.x == 0) resolve_scales(p, s_enc);
         __syncthreads();
     }
-    TensorEncoder kenc, venc;
-    if (kWrite) {
-        kenc = s_enc[0];
-        venc = s_enc[1];
+    if (early) {
+        // rows and table are in; the scales and every store wait
+        wait_for_previous_grid();
+        allow_next_grid();
     }
+    TensorEncoder kenc, venc;
+    if (kWrite) resolve_scales(p, kenc, venc);
 
     const bool small_slots = p.num_slots <= 0x7FFFFFFF;
     uint32_t kacc = 0, vacc = 0;
 
-    for (bool first = true; t < total; t += nwarps, first = false) {
-        if (!first) load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
+    // the first token (the only one unless the grid is smaller than the
+    // batch), then the rest of the grid-stride loop
+    if (t < total)
+        process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
+                                                            s_table, log2, small_slots, kacc,
+                                                            vacc);
+    for (t += nwarps; t < total; t += nwarps) {
+        load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
         process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
                                                             s_table, log2, small_slots, kacc,
                                                             vacc);
@@ -643,7 +692,6 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
 // rows go through the same code as a one-layer write.
 template <int kChunks>
 __global__ void __launch_bounds__(kKvThreads, 4) kv_write_layers_kernel(const KvLayers L) {
-    __shared__ TensorEncoder s_enc[2];
     const KvLayer &ly = L.layer[blockIdx.y];
     KvPass p;
     p.k = ly.k;
@@ -667,20 +715,22 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_write_layers_kernel(const Kv
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kKvThreads) >> 5;
     const int nchunks = kChunks > 0 ? kChunks : (p.elems >> 3);
-    if (warp < p.num_tokens && lane < 3) prefetch_row<false, true>(p, warp, lane);
+    if (warp < p.num_tokens && lane < 2) prefetch_row<false>(p, warp, lane);
     wait_for_previous_grid();
     allow_next_grid();
 
     Row r;
     int64_t t = warp;
     if (t < p.num_tokens) load_row<false, true, kChunks>(p, t, lane, nchunks, r);
-    if (threadIdx.x == 0) resolve_layer_scales(p, s_enc);
-    __syncthreads();
-    const TensorEncoder kenc = s_enc[0], venc = s_enc[1];
+    TensorEncoder kenc, venc;
+    resolve_layer_scales(p, kenc, venc);
     const bool small_slots = p.num_slots <= 0x7FFFFFFF;
     uint32_t kacc = 0, vacc = 0;
-    for (bool first = true; t < p.num_tokens; t += nwarps, first = false) {
-        if (!first) load_row<false, true, kChunks>(p, t, lane, nchunks, r);
+    if (t < p.num_tokens)
+        process_row<false, false, true, false, kChunks>(p, r, t, lane, nchunks, kenc, venc,
+                                                        nullptr, 0, small_slots, kacc, vacc);
+    for (t += nwarps; t < p.num_tokens; t += nwarps) {
+        load_row<false, true, kChunks>(p, t, lane, nchunks, r);
         process_row<false, false, true, false, kChunks>(p, r, t, lane, nchunks, kenc, venc,
                                                         nullptr, 0, small_slots, kacc, vacc);
     }
@@ -707,11 +757,6 @@ __global__ void calib_set_kernel(float *state, float a, float b, float c, float 
 // ---------------------------------------------------------------------------
 // launch geometry
 
-int table_log2_host(int64_t entries) {
-    int log2 = 6;
-    while ((int64_t{1} << log2) < 2 * entries) ++log2;
-    return log2;
-}
 
 struct DeviceInfo {
     int sms = 0;
@@ -805,7 +850,7 @@ cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
     auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, X, 64> : kv_pass_kernel<A, S, W, X, 0>;
     const int64_t tokens = p.num_tokens + (X ? p.x_tokens : 0);
     const int64_t wanted = (tokens + kKvWarps - 1) / kKvWarps;
-    const size_t smem = X ? (size_t{4} << table_log2_host(p.x_tokens)) : 0;
+    const size_t smem = X ? static_cast<size_t>(crossing_set_bytes(p.num_slots, p.x_tokens)) : 0;
     int grid = 1;
     cudaError_t e = grid_for(kernel, kKvThreads, smem, wanted, &grid);
     if (e != cudaSuccess) return e;

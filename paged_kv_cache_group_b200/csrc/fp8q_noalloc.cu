@@ -136,6 +136,9 @@ extern "C" FP8Q_API fp8q_status fp8_kv_calib_window_noalloc(
     w.cache_stride = cache_stride;
     w.num_slots = num_blocks * block_size;
     w.do_write = true;
+    // every pass below follows a launch of this call (calib_init first), and
+    // none reads what the launch before it writes
+    w.early_loads = true;
 
     const uint16_t *k16 = static_cast<const uint16_t *>(k);
     const uint16_t *v16 = static_cast<const uint16_t *>(v);

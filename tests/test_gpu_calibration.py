@@ -127,6 +127,22 @@ def test_crossing_batch_reuses_a_block_of_the_last_staged_batch(fused):
 
 
 @pytest.mark.parametrize("fused", [False, True])
+def test_crossing_set_of_a_pool_above_the_bitmap_limit(fused):
+    # the same window and block reuse in a pool of 19200 blocks (307200 slots,
+    # above the 2^18 slots a crossing bitmap covers): the merged launch keeps
+    # the crossing slots in its hash set instead
+    spec, batches, _ = workloads.calib_window(recycle={6: (2, 1), 9: (8, 1)})
+    big = workloads.PoolSpec(19200, spec.block_size, spec.heads, spec.dim)
+    assert big.num_slots > 2 ** 18
+    shift = 19000 * spec.block_size
+    moved = [workloads.KvBatchInput(b.k, b.v, b.slot_mapping + shift, b.key_stride,
+                                    b.value_stride) for b in batches]
+    g, c, steps = _run_both(big, moved, workloads.CALIB_WINDOW, 1.0, fused, check_every=False)
+    assert steps[8] == fp8q.STEP_FREEZE
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
 def test_crossing_batch_larger_than_one_merged_launch(fused):
     # 9000 tokens reach a 1-token window at once: above the merge limit, the
     # crossing batch gets a launch of its own after the scales are published
