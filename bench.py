@@ -493,6 +493,19 @@ def measure_targets(w: Workload, stream, args) -> dict:
                                     "vs_pages_h100_636_gbs": round(gbs / 636.0, 2),
                                     "launch": "single launch in its own graph"}
 
+    # the fixed cost of this way of timing one launch: the same quantizer on a
+    # single 128-element group (one CTA), in its own graph, timed the same way
+    x1 = w.x[:1, :128].contiguous()
+    q1 = torch.empty((1, 128), dtype=torch.uint8, device=w.device)
+    s1 = torch.empty((1, 1), dtype=torch.float32, device=w.device)
+
+    def gq1(mark):
+        fp8q.fp8_group_quant(x1, q1, s1)
+        mark(0)
+
+    out["launch_floor_1x128"] = {"us": round(timed(gq1, 1), 3),
+                                 "launch": "single launch in its own graph, one 128-element group"}
+
     # back to back over four distinct activations (as consecutive layers
     # quantize theirs): inputs and outputs 4 x 71 MB, more than L2 holds
     xs = [w.x] + [w.x.clone() for _ in range(3)]

@@ -9,17 +9,22 @@
 // Exact arithmetic.  A code is E4M3(fp32(x / s)).  The fp32 quotient is
 // formed from r = RN(1/s) (one IEEE reciprocal per group or per tensor) with
 // one product and one FMA correction:
-//     q0 = RN(x * r);  e = q0*s - x (exact in an FMA);  q = RN(q0 - e*r)
+//     q0 = RN(x * r);  e = x - q0*s (exact in an FMA);  q = RN(q0 + e*r)
 // By Markstein's theorem (r within half an ulp of 1/s, q0 within one ulp of
-// x/s, no underflow or overflow) q is the correctly rounded x/s.  Forming the
-// remainder as q0*s - x and subtracting it keeps the sign of a zero quotient:
-// for x = -0, q0 = -0, e = +0 and q = -0 - (+0)*r = -0.  For the activation
-// quantizer this was checked exhaustively over every pair of bf16 x and bf16
-// group maximum; for a per-tensor scale the fast form is used only while the
-// scale lies in [2^-64, 2^64] (x clamped so that x * r cannot overflow, which
-// only changes values that saturate anyway), and __fdiv_rn is used outside
-// that range.  The quotient is then rounded by the hardware conversion
-// cvt.rn.satfinite.e4m3x2.f32: nearest-even, saturating to +-448.
+// x/s, no underflow or overflow) q is the correctly rounded x/s.  The three
+// steps run on pairs of values (fma.rn.f32x2, two independent IEEE
+// operations per instruction).  This form can turn the quotient of x = -0
+// into +0, so after the conversion the sign bit of every code whose input is
+// negative is set again from the bf16 sign bits (a no-op for every other
+// negative input, whose code already carries it).  When s is a power of two,
+// r = 1/s exactly and RN(x * r) is already the quotient: one product.  For
+// the activation quantizer this was checked exhaustively over every pair of
+// bf16 x and bf16 group maximum; for a per-tensor scale the reciprocal form
+// is used only while the scale lies in [2^-64, 2^64] (x clamped so that x * r
+// cannot overflow, which only changes values that saturate anyway), and
+// __fdiv_rn is used outside that range.  The quotient is then rounded by the
+// hardware conversion cvt.rn.satfinite.e4m3x2.f32: nearest-even, saturating
+// to +-448.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -122,18 +127,64 @@ struct Divisor {
     float r;     // RN(1/s)
 };
 
-// Correctly rounded x / s (see the file comment).
-__device__ __forceinline__ float quotient(float x, const Divisor &d) {
-    const float q0 = __fmul_rn(x, d.r);
-    const float e = __fmaf_rn(q0, d.s, -x);
-    return __fmaf_rn(-e, d.r, q0);
+// A pair of fp32 values in one 64-bit register, as the f32x2 instructions take.
+__device__ __forceinline__ uint64_t pair(float lo, float hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ uint64_t pair_of_bf16x2(uint32_t w) { return pair(bf16_lo(w), bf16_hi(w)); }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// Two fp32 values (a pair) to two E4M3 codes: byte 0 <- lo, byte 1 <- hi.
+__device__ __forceinline__ uint32_t e4m3x2_pair(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return e4m3x2(lo, hi);
+}
+
+// The divisor as pairs: {r, r} and {-s, -s}.
+struct PairDivisor {
+    uint64_t r2, ns2;
+};
+__device__ __forceinline__ PairDivisor pair_divisor(const Divisor &d) {
+    return PairDivisor{pair(d.r, d.r), pair(-d.s, -d.s)};
+}
+
+// Correctly rounded quotients of a pair (see the file comment).
+__device__ __forceinline__ uint64_t quotient2(uint64_t x, const PairDivisor &d) {
+    const uint64_t q0 = mul2(x, d.r2);
+    const uint64_t e = fma2(q0, d.ns2, x);
+    return fma2(e, d.r2, q0);
+}
+
+// Codes of four values (bf16x2 words w0, w1) with the sign of every negative
+// input's code set from the bf16 sign bits.
+__device__ __forceinline__ uint32_t encode4(uint32_t w0, uint32_t w1, const PairDivisor &d) {
+    const uint32_t c = e4m3x2_pair(quotient2(pair_of_bf16x2(w0), d)) |
+                       (e4m3x2_pair(quotient2(pair_of_bf16x2(w1), d)) << 16);
+    return c | (__byte_perm(w0, w1, 0x7531) & 0x80808080u);
+}
+
+// Codes of four values for a power-of-two scale: r is exact, one product.
+__device__ __forceinline__ uint32_t encode4_pow2(uint32_t w0, uint32_t w1, uint64_t r2) {
+    return e4m3x2_pair(mul2(pair_of_bf16x2(w0), r2)) |
+           (e4m3x2_pair(mul2(pair_of_bf16x2(w1), r2)) << 16);
 }
 
 // Group scale RN(y / 448) for y >= 1e-12.  448 = 7 * 64, so the quotient is
 // RN(y / 7) * 2^-6 exactly (no underflow in that range), and RN(y / 7) is the
 // correctly rounded division by the constant 7 from RN(1/7), by the same
-// Markstein step as above.  Checked against IEEE division for every bf16
-// group maximum.
+// Markstein step as above.  Checked against IEEE division for every fp32 y
+// from 1e-12 to the largest finite value.
 __device__ __forceinline__ float group_scale(float y) {
     constexpr float kRecip7 = 0x1.24924ap-3f;   // RN(1/7)
     const float q0 = __fmul_rn(y, kRecip7);
@@ -141,13 +192,12 @@ __device__ __forceinline__ float group_scale(float y) {
     return __fmul_rn(__fmaf_rn(-e, kRecip7, q0), 0x1p-6f);
 }
 
-__device__ __forceinline__ uint2 encode8(const uint4 &w, const Divisor &d) {
-    uint2 o;
-    o.x = e4m3x2(quotient(bf16_lo(w.x), d), quotient(bf16_hi(w.x), d)) |
-          (e4m3x2(quotient(bf16_lo(w.y), d), quotient(bf16_hi(w.y), d)) << 16);
-    o.y = e4m3x2(quotient(bf16_lo(w.z), d), quotient(bf16_hi(w.z), d)) |
-          (e4m3x2(quotient(bf16_lo(w.w), d), quotient(bf16_hi(w.w), d)) << 16);
-    return o;
+__device__ __forceinline__ uint2 encode8(const uint4 &w, const PairDivisor &d) {
+    return make_uint2(encode4(w.x, w.y, d), encode4(w.z, w.w, d));
+}
+
+__device__ __forceinline__ uint2 encode8_pow2(const uint4 &w, uint64_t r2) {
+    return make_uint2(encode4_pow2(w.x, w.y, r2), encode4_pow2(w.z, w.w, r2));
 }
 
 // IEEE division per element, for scales outside the fast range.
@@ -169,12 +219,14 @@ struct TensorEncoder {
     Divisor d;
     uint32_t lo2, hi2;   // clamp bounds as bf16x2 (-T, T)
     bool fast;
+    bool pow2;           // s is a power of two: RN(x * r) is the quotient
     bool clamp;
     bool ok;             // scale is a positive number
 
     __device__ __forceinline__ void init(float s) {
         ok = s > 0.0f;   // false for NaN
         fast = (s >= 0x1p-64f) && (s <= 0x1p64f);
+        pow2 = fast && (__float_as_uint(s) & 0x7FFFFFu) == 0;
         d.s = s;
         d.r = __frcp_rn(s);
         clamp = d.r > 1.0f;
@@ -193,11 +245,17 @@ struct TensorEncoder {
         return w;
     }
 
-    // Two chunks of a row.  Only magnitudes at or beyond T can overflow
-    // x * r, and T is far above any realistic K/V, so the clamp runs only
-    // when the pair's largest magnitude reaches it.
+    // Two chunks of a row.  Power-of-two scale: one product per value (an
+    // overflow to infinity saturates like the quotient it stands for).
+    // Otherwise only magnitudes at or beyond T can overflow x * r, and T is
+    // far above any realistic K/V, so the clamp runs only when the pair's
+    // largest magnitude reaches it.
     __device__ __forceinline__ void encode2(uint4 a, uint4 b, uint2 &oa, uint2 &ob) const {
-        if (fast) {
+        if (pow2) {
+            const uint64_t r2 = pair(d.r, d.r);
+            oa = encode8_pow2(a, r2);
+            ob = encode8_pow2(b, r2);
+        } else if (fast) {
             if (clamp) {
                 const uint32_t m = absmax_bits16(absmax_uint4(absmax_uint4(0u, a), b));
                 if (m >= (hi2 & 0xFFFFu)) {
@@ -205,8 +263,9 @@ struct TensorEncoder {
                     b = clamp4(b, lo2, hi2);
                 }
             }
-            oa = encode8(a, d);
-            ob = encode8(b, d);
+            const PairDivisor pd = pair_divisor(d);
+            oa = encode8(a, pd);
+            ob = encode8(b, pd);
         } else {
             oa = encode8_div(a, d.s);
             ob = encode8_div(b, d.s);
@@ -285,11 +344,12 @@ group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
         const bool valid = g < total_groups;
         uint4 c[4];
         const Divisor d = quant_group_load(group_src(valid ? g : 0), valid, ql, c);
+        const PairDivisor pd = pair_divisor(d);
         if (valid) {
             uint8_t *dst = q + g * 128;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) = encode8(c[j], d);
+                *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) = encode8(c[j], pd);
             if (ql == 0) scales[g] = d.s;
         }
     }
@@ -327,12 +387,13 @@ group_quant_kmajor_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
         uint4 c[4];
         const Divisor d =
             quant_group_load(x + (live ? row * x_row_stride + col * 128 : 0), live, ql, c);
+        const PairDivisor pd = pair_divisor(d);
         if (row < m_pad) {
             uint8_t *dst = q + row * k + col * 128;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) =
-                    live ? encode8(c[j], d) : make_uint2(0, 0);
+                    live ? encode8(c[j], pd) : make_uint2(0, 0);
             if (ql == 0) scales_km[col * m_pad + row] = live ? d.s : 0.0f;
         }
     }
