@@ -854,12 +854,16 @@ def run_profile(args) -> None:
     """A few eager steps on `--layers` layers for an ncu capture: each step is
     the bench step (group quant, then per layer the calibrating write) followed
     by the steady-state write of every layer one launch each, then the same as
-    one fp8_kv_write_layers launch.  Select kernels with ncu -k / -s / -c.
+    one fp8_kv_write_layers launch, then the activation quantized K-major for a
+    GEMM padded to ceil16(M) rows.  Select kernels with ncu -k / -s / -c.
     ncu flushes caches itself, so no flush buffers are allocated."""
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = Workload(dev, args.layers, flush=False)
     scale = torch.tensor([0.05, 0.05], dtype=torch.float32, device=dev)
+    m_pad = w.fp8q.ceil16(M)
+    qk = torch.empty((m_pad, K), dtype=torch.uint8, device=dev)
+    sk = torch.empty((K // 128, m_pad), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         for i in range(args.warmup + args.steps):
@@ -870,6 +874,7 @@ def run_profile(args) -> None:
                                     scale_dev=scale)
             w.fp8q.fp8_kv_write_layers(w.k, w.v, w.slots, w.k_pool, w.v_pool,
                                        scale_devs=[scale] * w.layers)
+            w.fp8q.fp8_group_quant_kmajor(w.x, m_pad, qk, sk)
     torch.cuda.synchronize()
     assert w.fp8q.fp8q_device_error(clear=True) == 0
     print(json.dumps({"profile": "done", "layers": args.layers,

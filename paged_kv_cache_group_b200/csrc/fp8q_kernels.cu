@@ -328,14 +328,23 @@ group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kGqThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGqThreads) >> 5;
     const int64_t octets = (total_groups + 7) >> 3;
+    // Strided rows: this lane's group as (row, column), advanced by the grid's
+    // stride without a division per step.
+    const int64_t g0 = warp * 8 + sub;
+    int64_t row = kPacked ? 0 : g0 / groups_per_row;
+    int64_t col = kPacked ? 0 : g0 - row * groups_per_row;
+    const int64_t step = nwarps * 8;
+    const int64_t drow = kPacked ? 0 : step / groups_per_row;
+    const int64_t dcol = kPacked ? 0 : step - drow * groups_per_row;
     auto group_src = [&](int64_t g) -> const uint16_t * {
         if (kPacked) return x + g * 128;
-        const uint64_t row = static_cast<uint64_t>(g) / groups_per_row;
-        return x + row * x_row_stride + (static_cast<uint64_t>(g) - row * groups_per_row) * 128;
+        return x + row * x_row_stride + col * 128;
     };
     // the first eight groups this warp reads: one 256-byte group per lane 0..7
-    if (lane < 8 && warp < octets && warp * 8 + lane < total_groups)
-        prefetch_l2_bulk(group_src(warp * 8 + lane), 256);
+    if (kPacked && lane < 8 && warp < octets && warp * 8 + lane < total_groups)
+        prefetch_l2_bulk(x + (warp * 8 + lane) * 128, 256);
+    if (!kPacked && (lane & 3) == 0 && warp < octets && g0 < total_groups)
+        prefetch_l2_bulk(group_src(g0), 256);
     wait_for_previous_grid();
     allow_next_grid();
 
@@ -343,7 +352,7 @@ group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
         const int64_t g = o * 8 + sub;
         const bool valid = g < total_groups;
         uint4 c[4];
-        const Divisor d = quant_group_load(group_src(valid ? g : 0), valid, ql, c);
+        const Divisor d = quant_group_load(valid ? group_src(g) : x, valid, ql, c);
         const PairDivisor pd = pair_divisor(d);
         if (valid) {
             uint8_t *dst = q + g * 128;
@@ -351,6 +360,14 @@ group_quant_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
             for (int j = 0; j < 4; ++j)
                 *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) = encode8(c[j], pd);
             if (ql == 0) scales[g] = d.s;
+        }
+        if (!kPacked) {
+            row += drow;
+            col += dcol;
+            if (col >= groups_per_row) {
+                col -= groups_per_row;
+                ++row;
+            }
         }
     }
 }
@@ -371,17 +388,20 @@ group_quant_kmajor_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGqThreads) >> 5;
     const int64_t octets = ((m_pad + 7) >> 3) * groups_per_row;
     const int64_t k = static_cast<int64_t>(groups_per_row) * 128;
+    // this warp's (row octet, column), advanced by the grid's stride without
+    // a division per step
+    int64_t ro = warp / groups_per_row;
+    int64_t col = warp - ro * groups_per_row;
+    const int64_t dro = nwarps / groups_per_row;
+    const int64_t dcol = nwarps - dro * groups_per_row;
     if (lane < 8 && warp < octets) {
-        const int64_t ro = warp / groups_per_row;
         const int64_t row = ro * 8 + lane;
-        if (row < m) prefetch_l2_bulk(x + row * x_row_stride + (warp - ro * groups_per_row) * 128, 256);
+        if (row < m) prefetch_l2_bulk(x + row * x_row_stride + col * 128, 256);
     }
     wait_for_previous_grid();
     allow_next_grid();
 
     for (int64_t o = warp; o < octets; o += nwarps) {
-        const int64_t ro = o / groups_per_row;
-        const int64_t col = o - ro * groups_per_row;
         const int64_t row = ro * 8 + sub;
         const bool live = row < m;
         uint4 c[4];
@@ -395,6 +415,12 @@ group_quant_kmajor_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
                 *reinterpret_cast<uint2 *>(dst + (ql + 4 * j) * 8) =
                     live ? encode8(c[j], pd) : make_uint2(0, 0);
             if (ql == 0) scales_km[col * m_pad + row] = live ? d.s : 0.0f;
+        }
+        ro += dro;
+        col += dcol;
+        if (col >= groups_per_row) {
+            col -= groups_per_row;
+            ++ro;
         }
     }
 }
