@@ -683,11 +683,20 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     // a CTA whose first token is a crossing token never sees a staged one.
     const bool need_table =
         kCross && static_cast<int64_t>(blockIdx.x) * kKvWarps < p.num_tokens;
+    // The plain write takes two tokens per warp (half the grid, so the next
+    // launch's CTAs fit beside this one's and can prefetch early); both rows
+    // are prefetched before the wait and loaded together.
+    constexpr bool kTwo = kWrite && !kAmax && !kStage && !kCross;
     const bool early = p.early_loads;
     if (!early) {
         // the first token's K row, V row and slot into L2 while the previous
         // kernel finishes (and, for a merged crossing batch, its slot list)
-        if (warp < total && lane < 2) prefetch_row<kCross>(p, warp, lane);
+        if (kTwo) {
+            const int64_t tt = warp + (lane >> 1) * nwarps;
+            if (lane < 4 && tt < total) prefetch_row<kCross>(p, tt, lane & 1);
+        } else if (warp < total && lane < 2) {
+            prefetch_row<kCross>(p, warp, lane);
+        }
         if (need_table && threadIdx.x == 32) {
             const int64_t bytes = p.x_tokens * 8;
             if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0)
@@ -739,10 +748,21 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
 
     // the first token (the only one unless the grid is smaller than the
     // batch), then the rest of the grid-stride loop
-    if (t < total)
+    if (kTwo && t + nwarps < total) {
+        Row r2;
+        load_row<kCross, kSlot, kChunks>(p, t + nwarps, lane, nchunks, r2);
         process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
                                                             s_table, log2, small_slots, kacc,
                                                             vacc);
+        t += nwarps;
+        process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r2, t, lane, nchunks, kenc, venc,
+                                                            s_table, log2, small_slots, kacc,
+                                                            vacc);
+    } else if (t < total) {
+        process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
+                                                            s_table, log2, small_slots, kacc,
+                                                            vacc);
+    }
     for (t += nwarps; t < total; t += nwarps) {
         load_row<kCross, kSlot, kChunks>(p, t, lane, nchunks, r);
         process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
@@ -936,7 +956,8 @@ template <bool A, bool S, bool W, bool X>
 cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
     auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, X, 64> : kv_pass_kernel<A, S, W, X, 0>;
     const int64_t tokens = p.num_tokens + (X ? p.x_tokens : 0);
-    const int64_t wanted = (tokens + kKvWarps - 1) / kKvWarps;
+    const int64_t per_cta = (W && !A && !S && !X) ? 2 * kKvWarps : kKvWarps;   // see kTwo
+    const int64_t wanted = (tokens + per_cta - 1) / per_cta;
     const size_t smem = X ? static_cast<size_t>(crossing_set_bytes(p.num_slots, p.x_tokens)) : 0;
     int grid = 1;
     cudaError_t e = grid_for(kernel, kKvThreads, smem, wanted, &grid);
