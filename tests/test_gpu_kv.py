@@ -77,6 +77,13 @@ def test_large_layer_full_pool():
     _parity(spec, b, np.float32(20.0) / np.float32(448.0), np.float32(2.0))
 
 
+def test_batch_longer_than_two_tokens_per_warp_of_a_full_grid():
+    # 20000 tokens: more than two per warp of the largest resident grid, so the
+    # plain write's grid-stride loop runs after its two-token start
+    spec = workloads.large_kv_spec()
+    _parity(spec, workloads.large_kv_layer(11, tokens=20000), 0.05, 0.07)
+
+
 def test_padded_cache_stride_and_wide_rows():
     spec = workloads.PoolSpec(24, 8, 8, 128)          # E = 1024: two chunk rounds per warp
     g = workloads.generator(600, 0, 0)
