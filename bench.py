@@ -284,6 +284,34 @@ def time_graph(w: Workload, stream, graph, reps: int, reset_state: bool) -> list
     return out
 
 
+def drained_step_ms(w: Workload, stream, graph, reps: int) -> float:
+    """Step time with the write-back of its dirty L2 lines included.  The step
+    leaves up to an L2's worth of written lines dirty; the untimed flush before
+    the next step writes them back.  Here each step is followed, inside the
+    timed region, by a read of a clean 2x-L2 buffer that evicts them, and the
+    same read after a clean L2 (no dirty lines) is subtracted."""
+    drain = torch.ones_like(w.flush_read)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with_wb, without = [], []
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            w.reset(i)
+            start.record()
+            graph.replay()
+            sink = torch.amax(drain)
+            end.record()
+            end.synchronize()
+            with_wb.append(start.elapsed_time(end))
+            w.reset(i)
+            start.record()
+            sink = torch.amax(drain)
+            end.record()
+            end.synchronize()
+            without.append(start.elapsed_time(end))
+    del drain, sink
+    return statistics.mean(with_wb) - statistics.mean(without)
+
+
 def kernel_sequences(w: Workload, stream, reps: int) -> dict:
     """Average launch duration of each kernel of the step, from a graph of its
     launches exactly as the step issues them (one per layer, back to back),
@@ -396,6 +424,7 @@ def run_native(args, dist: Dist) -> dict | None:
             end.synchronize()
             eager_ms.append(start.elapsed_time(end))
 
+    drained_ms = drained_step_ms(w, stream, graph, reps=max(20, min(args.steps, 200)))
     seq = kernel_sequences(w, stream, reps=max(5, min(args.steps, 50)))
     targets = measure_targets(w, stream, args)
     e2e = None if args.no_e2e else measure_e2e(w, stream, args)
@@ -448,6 +477,13 @@ def run_native(args, dist: Dist) -> dict | None:
             "kernels": kernels,
             "targets": targets,
             "eager_ms_per_step": round(statistics.median(eager_ms), 4),
+            "writeback_drained": {
+                "ms_per_step": round(drained_ms, 5),
+                "value": round(step_bytes(args.layers) / (drained_ms * 1e-3) / 1e9, 2),
+                "unit": "GB/s",
+                "method": ("rank 0: (step + read of a clean 2x-L2 buffer) - (the same read on a "
+                           "clean L2): the step with the write-back of the dirty L2 lines it "
+                           "leaves behind counted in its time")},
             "gpu_launches": gpu_launches,
             "clocks": clock_info,
         }
