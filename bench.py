@@ -746,7 +746,18 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
     s = statistics.median(times)
     return {"value": round(sample_bytes() / s / 1e9, 4), "unit": "GB/s", "cores": 1,
             "kind": "oracle", "sample": SAMPLE_DESC, "repeats": len(times),
-            "host_cores": os.cpu_count()}
+            "host_cores": os.cpu_count(), "cpu_model": cpu_model()}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args) -> dict | None:
