@@ -208,7 +208,30 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
 
     int64_t rewritten = 0;
     bool published = false;
-    if (merge && last < 0) {
+
+    // Two or more staged batches with rows: every staged row and the crossing
+    // batch in one launch, each slot written by its last writer in arrival
+    // order, when the window is small enough for the last-writer table.
+    int64_t with_rows = 0;
+    for (const StagedBatch &b : c->batches) with_rows += b.num_tokens > 0;
+    const int64_t whole_rows = c->used_tokens + (merge ? crossing->num_tokens : 0);
+    if (with_rows >= 2 && whole_rows <= fp8q::kMaxLastWriterTokens &&
+        p.num_slots <= 0x7FFFFFFF) {
+        KvPass q = merge ? with_crossing(p) : p;
+        q.k = c->stage_k;
+        q.v = c->stage_v;
+        q.slot_mapping = c->stage_slots;
+        q.num_tokens = c->used_tokens;
+        q.last_writer = true;
+        if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
+        rewritten = c->used_tokens;
+        published = true;
+        if (crossing != nullptr && !merge) {
+            KvPass x = *crossing;
+            x.early_loads = chained;
+            if (fp8q::launch_kv_pass(x, stream) != cudaSuccess) return FP8Q_ECUDA;
+        }
+    } else if (merge && last < 0) {
         // nothing staged with rows: the crossing batch alone, publishing the scales
         KvPass q = with_crossing(p);
         q.num_tokens = 0;

@@ -75,6 +75,11 @@ struct KvPass {
     // produced by the previous kernel and the stores wait.  Set only where a
     // call enqueues that whole chain itself.
     bool early_loads = false;
+    // Replay of a whole window in one launch: rows [0, num_tokens) are every
+    // staged batch in arrival order and the crossing rows follow; a row is
+    // written only if no later row of the launch has the same slot.  Needs
+    // num_tokens + x_tokens <= kMaxLastWriterTokens.
+    bool last_writer = false;
 };
 
 // Several layers' writes in one launch (fp8_kv_write_layers): row strides,
@@ -117,6 +122,7 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream);
 // Largest crossing batch a single launch can merge with a replay (its slots
 // go into a hash set in shared memory); larger ones use two launches.
 constexpr int64_t kMaxMergedCrossing = 8192;
+constexpr int64_t kMaxLastWriterTokens = 2048;
 bool can_merge_crossing(const KvPass &p);
 
 // Group quantization with phantom rows m..m_pad-1 zeroed and the scales

@@ -497,6 +497,50 @@ __device__ __forceinline__ bool crossing_contains(const uint32_t *tab, int log2,
     return table_contains(tab, log2, key);
 }
 
+// Last-writer table of a whole-window replay: 2^L slot keys followed by 2^L
+// values, the value of a slot being 1 + the highest row index that writes it
+// (open addressing, linear probing, at most half full).
+__host__ __device__ __forceinline__ int last_writer_log2(int64_t rows) {
+    int log2 = 6;
+    while ((int64_t{1} << log2) < 2 * rows) ++log2;
+    return log2;
+}
+
+__device__ __forceinline__ void last_writer_insert(uint32_t *tab, int log2, uint32_t key,
+                                                   uint32_t row1) {
+    const uint32_t mask = (1u << log2) - 1u;
+    uint32_t h = slot_hash(key, log2);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {   // bounded: the table is never full
+        const uint32_t prev = atomicCAS(&tab[h], kEmptySlot, key);
+        if (prev == kEmptySlot || prev == key) {
+            atomicMax(&tab[(1u << log2) + h], row1);
+            return;
+        }
+        h = (h + 1u) & mask;
+    }
+}
+
+__device__ __forceinline__ uint32_t last_writer_of(const uint32_t *tab, int log2, uint32_t key) {
+    const uint32_t mask = (1u << log2) - 1u;
+    uint32_t h = slot_hash(key, log2);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+        const uint32_t v = tab[h];
+        if (v == key) return tab[(1u << log2) + h];
+        if (v == kEmptySlot) return 0;
+        h = (h + 1u) & mask;
+    }
+    return 0;
+}
+
+// Whether a later row of the launch writes this row's slot.  log2 < 0: the
+// last-writer table of a whole-window replay (2^-log2 entries); otherwise the
+// crossing set, which only staged rows consult.
+__device__ __forceinline__ bool superseded(const uint32_t *tab, int log2, uint32_t key, int64_t t,
+                                           int64_t num_tokens) {
+    if (log2 < 0) return last_writer_of(tab, -log2, key) != static_cast<uint32_t>(t + 1);
+    return t < num_tokens && crossing_contains(tab, log2, key);
+}
+
 // Scales of a write pass (see KvPass).  Every warp resolves them itself from
 // two loads issued together with its row loads; a CTA-wide broadcast through
 // shared memory would put a barrier behind the slowest of those loads.  Lane 0
@@ -594,8 +638,8 @@ __device__ __forceinline__ void process_row(const KvPass &p, Row &r, int64_t t, 
     if (kWrite && slot >= 0) {
         if (slot >= p.num_slots) {
             if (lane == 0) atomicOr(&g_error_word, kErrSlot);
-        } else if (!(kCross && t < p.num_tokens &&
-                     crossing_contains(table, log2, static_cast<uint32_t>(slot)))) {
+        } else if (!(kCross && superseded(table, log2, static_cast<uint32_t>(slot), t,
+                                          p.num_tokens))) {
             int64_t blk, off;
             if (p.block_shift >= 0) {
                 blk = slot >> p.block_shift;
@@ -688,8 +732,9 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     // Only CTAs that rewrite staged tokens consult the crossing slots.  With
     // the grid-stride loop a CTA's tokens are blockIdx.x*8 + k*nwarps + w, so
     // a CTA whose first token is a crossing token never sees a staged one.
+    // A whole-window replay checks every row against its last-writer table.
     const bool need_table =
-        kCross && static_cast<int64_t>(blockIdx.x) * kKvWarps < p.num_tokens;
+        kCross && (p.last_writer || static_cast<int64_t>(blockIdx.x) * kKvWarps < p.num_tokens);
     // The plain write takes two tokens per warp (half the grid, so the next
     // launch's CTAs fit beside this one's and can prefetch early); both rows
     // are prefetched before the wait and loaded together.
@@ -706,8 +751,15 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
         }
         if (need_table && threadIdx.x == 32) {
             const int64_t bytes = p.x_tokens * 8;
-            if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0)
+            if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0 &&
+                bytes > 0)
                 prefetch_l2_bulk(p.x_slots, static_cast<uint32_t>(bytes));
+        }
+        if (kCross && p.last_writer && threadIdx.x == 64) {
+            const int64_t bytes = p.num_tokens * 8;
+            if ((reinterpret_cast<uintptr_t>(p.slot_mapping) & 15) == 0 && bytes % 16 == 0 &&
+                bytes > 0)
+                prefetch_l2_bulk(p.slot_mapping, static_cast<uint32_t>(bytes));
         }
         wait_for_previous_grid();
         allow_next_grid();
@@ -721,7 +773,24 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     // 2. per CTA: the crossing slots, as a bitmap over the pool's slots or,
     // for larger pools, a hash set
     int log2 = 0;
-    if (need_table) {
+    if (need_table && p.last_writer) {
+        const int lw = last_writer_log2(total);
+        log2 = -lw;
+        uint4 *tab4 = reinterpret_cast<uint4 *>(s_table);
+        const int keys4 = (1 << lw) / 4;
+        const uint4 empty = make_uint4(kEmptySlot, kEmptySlot, kEmptySlot, kEmptySlot);
+        for (int i = threadIdx.x; i < 2 * keys4; i += kKvThreads)
+            tab4[i] = i < keys4 ? empty : make_uint4(0, 0, 0, 0);
+        __syncthreads();
+        for (int64_t i = threadIdx.x; i < total; i += kKvThreads) {
+            const int64_t sl = i < p.num_tokens ? __ldg(p.slot_mapping + i)
+                                                : __ldg(p.x_slots + (i - p.num_tokens));
+            if (sl >= 0 && sl < p.num_slots)
+                last_writer_insert(s_table, lw, static_cast<uint32_t>(sl),
+                                   static_cast<uint32_t>(i + 1));
+        }
+        __syncthreads();
+    } else if (need_table) {
         const bool bitmap = p.num_slots <= kBitmapMaxSlots;
         log2 = bitmap ? 0 : table_log2(p.x_tokens);
         uint4 *tab4 = reinterpret_cast<uint4 *>(s_table);
@@ -965,7 +1034,10 @@ cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
     const int64_t tokens = p.num_tokens + (X ? p.x_tokens : 0);
     const int64_t per_cta = (W && !A && !S && !X) ? 2 * kKvWarps : kKvWarps;   // see kTwo
     const int64_t wanted = (tokens + per_cta - 1) / per_cta;
-    const size_t smem = X ? static_cast<size_t>(crossing_set_bytes(p.num_slots, p.x_tokens)) : 0;
+    const size_t smem =
+        !X ? 0
+           : p.last_writer ? (size_t{8} << last_writer_log2(tokens))
+                           : static_cast<size_t>(crossing_set_bytes(p.num_slots, p.x_tokens));
     int grid = 1;
     cudaError_t e = grid_for(kernel, kKvThreads, smem, wanted, &grid);
     if (e != cudaSuccess) return e;
@@ -1010,6 +1082,14 @@ bool can_merge_crossing(const KvPass &p) {
 
 cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
     const bool publish = p.do_write && p.freeze_amax != nullptr && p.scale_out != nullptr;
+    if (p.last_writer) {
+        if (!p.do_write || p.do_amax || p.do_stage || p.num_slots > 0x7FFFFFFF ||
+            p.num_tokens + p.x_tokens > kMaxLastWriterTokens ||
+            (p.x_tokens > 0 && p.x_slots == nullptr))
+            return cudaErrorInvalidValue;
+        if (p.num_tokens + p.x_tokens == 0 && p.scale_out == nullptr) return cudaSuccess;
+        return launch_kv_variant<false, false, true, true>(p, stream);
+    }
     const bool cross = p.do_write && p.x_tokens > 0;
     if (cross) {
         if (!can_merge_crossing(p) || p.do_amax || p.do_stage) return cudaErrorInvalidValue;

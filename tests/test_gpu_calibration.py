@@ -143,6 +143,22 @@ def test_crossing_set_of_a_pool_above_the_bitmap_limit(fused):
 
 
 @pytest.mark.parametrize("fused", [False, True])
+def test_whole_window_replay_with_a_block_written_four_times(fused):
+    # batch 1's block goes to batch 4, then to batch 7, then to the crossing
+    # batch 9: four writers of the same slots across the window.  The staged
+    # batches and the crossing batch replay in one launch, where each slot must
+    # end with its last writer.
+    spec, batches, blocks = workloads.calib_window(recycle={4: (1, 0), 7: (4, 0), 9: (7, 0)})
+    assert blocks[0][0] == blocks[3][0] == blocks[6][0] == blocks[8][0]
+    launches = fp8q.launch_count()
+    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused)
+    assert steps == [fp8q.STEP_STAGE] * 8 + [fp8q.STEP_FREEZE] + [fp8q.STEP_FROZEN] * 2
+    if fused:   # init, 8 in-window passes, absmax + one replay, 2 frozen writes
+        assert fp8q.launch_count() - launches == 1 + 8 + 2 + 2
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
 def test_crossing_batch_larger_than_one_merged_launch(fused):
     # 9000 tokens reach a 1-token window at once: above the merge limit, the
     # crossing batch gets a launch of its own after the scales are published
