@@ -159,6 +159,19 @@ def test_whole_window_replay_with_a_block_written_four_times(fused):
 
 
 @pytest.mark.parametrize("fused", [False, True])
+def test_whole_window_replay_then_a_crossing_batch_above_the_merge_limit(fused):
+    # two staged batches of 1000 tokens replay in one launch (no crossing rows
+    # in it); the 9000-token batch that reaches the 2048-token window is too
+    # large to merge and gets its own launch after the scales are published
+    spec = workloads.large_kv_spec()
+    full = workloads.large_kv_layer(12, tokens=11000)
+    chunks = workloads.split_batch(full, (1000, 1000, 9000))
+    g, c, steps = _run_both(spec, chunks, 2048, 1.0, fused, check_every=False)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
 def test_crossing_batch_larger_than_one_merged_launch(fused):
     # 9000 tokens reach a 1-token window at once: above the merge limit, the
     # crossing batch gets a launch of its own after the scales are published
