@@ -178,6 +178,28 @@ extern "C" FP8Q_API fp8q_status fp8_kv_calib_window_noalloc(
             r.freeze_amax = reinterpret_cast<uint32_t *>(state);
             r.headroom = h;
             r.scale_out = state + 2;
+            int32_t with_rows = 0;
+            for (int32_t s2 = 0; s2 < b; ++s2) with_rows += batch_tokens[s2] > 0;
+            if (with_rows >= 2 && n > 0 && staged + n <= fp8q::kMaxLastWriterTokens &&
+                w.num_slots <= 0x7FFFFFFF) {
+                // ... all of it in one launch, the crossing batch's rows last and
+                // every slot written by its last writer
+                fp8q::KvPass q = r;
+                q.k = stage_k;
+                q.v = stage_v;
+                q.slot_mapping = stage_slots;
+                q.num_tokens = staged;
+                q.xk = p.k;
+                q.xv = p.v;
+                q.x_key_stride = key_stride;
+                q.x_value_stride = value_stride;
+                q.x_slots = p.slot_mapping;
+                q.x_tokens = n;
+                q.last_writer = true;
+                if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
+                row += n;
+                continue;
+            }
             bool published = false;
             int64_t off = 0;
             for (int32_t s = 0; s < b; ++s) {
