@@ -49,10 +49,15 @@ def _bf16_rows(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must have a row dimension and at least one more")
     rows = t.shape[0]
     inner = 1
-    for size, stride in zip(reversed(t.shape[1:]), reversed(t.stride()[1:])):
-        if size != 1 and stride != inner:
-            raise ValueError(f"{name} rows must be contiguous")
+    for size in t.shape[1:]:
         inner *= size
+    if t.numel() == 0:          # no data: any strides (an empty array may carry zeros)
+        return rows, inner, inner
+    expect = 1
+    for size, stride in zip(reversed(t.shape[1:]), reversed(t.stride()[1:])):
+        if size != 1 and stride != expect:
+            raise ValueError(f"{name} rows must be contiguous")
+        expect *= size
     return rows, (t.stride(0) if rows > 1 else inner), inner
 
 
