@@ -87,3 +87,33 @@ def test_random_group_quant_both_layouts(i):
     assert np.array_equal(gqk, qk_ref), first_mismatch(gqk, qk_ref)
     assert np.array_equal(f32_bits(gsk), f32_bits(sk_ref)), first_mismatch(f32_bits(gsk),
                                                                            f32_bits(sk_ref))
+
+
+N_CALIB_CASES = 24
+
+
+def _calib_case(i: int):
+    g = workloads.generator(702, i, 0)
+    n = int(g.integers(2, 15))
+    sizes = [int(g.integers(1, 65)) for _ in range(n)]
+    nblk = [-(-t // 16) for t in sizes]
+    recycle = {}
+    for b in range(2, n + 1):
+        if g.random() < 0.3:
+            src = int(g.integers(1, b))
+            recycle[b] = (src, int(g.integers(0, nblk[src - 1])))
+    window = int(g.integers(1, sum(sizes) + 40))
+    headroom = float(g.choice([0.5, 1.0, 1.0, 1.25, 2.0]))
+    return tuple(sizes), recycle, window, headroom
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("i", range(N_CALIB_CASES))
+def test_random_calibration_windows(i, fused):
+    from test_gpu_calibration import _assert_frozen_state, _run_both
+    sizes, recycle, window, headroom = _calib_case(i)
+    spec, batches, _ = workloads.calib_window(batch_sizes=sizes, recycle=recycle)
+    g, c, steps = _run_both(spec, batches, window, headroom, fused)
+    if fp8q.STEP_FREEZE in steps:
+        _assert_frozen_state(g, c)
+    assert fp8q.fp8q_device_error(clear=True) == 0

@@ -215,7 +215,7 @@ def calib_window(batch_sizes=CALIB_BATCHES, row_pad: int = 0, recycle=None):
             sgn = np.where(g.random(rows.shape) < 0.5, -1.0, 1.0).astype(np.float32)
             rows[hit] = (mag * sgn)[hit]
             x.append(rows)
-        if b == 3:
+        if b == 3 and t > 5:
             x[0][5, 77] = np.float32(600.0)
         kb, vb = (to_bf16_bits(r) for r in x)
         if row_pad:
