@@ -718,13 +718,19 @@ __device__ __forceinline__ void prefetch_row(const KvPass &p, int64_t t, int lan
 
 // kChunks: 16-byte chunks per row when fixed at compile time (64 for the
 // common 4 x 128 rows), or 0 for any multiple of 8 elements.
-template <bool kAmax, bool kStage, bool kWrite, bool kCross, int kChunks>
-__global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) {
+//
+// kThreads: 256, or 512 for the merged freeze launch (kCross), where half as
+// many CTAs build the crossing slots' table (measured: 4.81 -> 4.44 us per
+// 4593-token replay; the other passes are faster with 256).
+template <bool kAmax, bool kStage, bool kWrite, bool kCross, int kChunks,
+          int kThreads = kKvThreads>
+__global__ void __launch_bounds__(kThreads, 1024 / kThreads) kv_pass_kernel(const KvPass p) {
+    constexpr int kWarps = kThreads / 32;
     extern __shared__ uint32_t s_table[];        // crossing slots (kCross)
 
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kKvThreads) >> 5;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int nchunks = kChunks > 0 ? kChunks : (p.elems >> 3);
     const int64_t total = p.num_tokens + (kCross ? p.x_tokens : 0);
     constexpr bool kSlot = kWrite || kStage;
@@ -734,7 +740,7 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     // a CTA whose first token is a crossing token never sees a staged one.
     // A whole-window replay checks every row against its last-writer table.
     const bool need_table =
-        kCross && (p.last_writer || static_cast<int64_t>(blockIdx.x) * kKvWarps < p.num_tokens);
+        kCross && (p.last_writer || static_cast<int64_t>(blockIdx.x) * kWarps < p.num_tokens);
     // The plain write takes two tokens per warp (half the grid, so the next
     // launch's CTAs fit beside this one's and can prefetch early); both rows
     // are prefetched before the wait and loaded together.
@@ -779,10 +785,10 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
         uint4 *tab4 = reinterpret_cast<uint4 *>(s_table);
         const int keys4 = (1 << lw) / 4;
         const uint4 empty = make_uint4(kEmptySlot, kEmptySlot, kEmptySlot, kEmptySlot);
-        for (int i = threadIdx.x; i < 2 * keys4; i += kKvThreads)
+        for (int i = threadIdx.x; i < 2 * keys4; i += kThreads)
             tab4[i] = i < keys4 ? empty : make_uint4(0, 0, 0, 0);
         __syncthreads();
-        for (int64_t i = threadIdx.x; i < total; i += kKvThreads) {
+        for (int64_t i = threadIdx.x; i < total; i += kThreads) {
             const int64_t sl = i < p.num_tokens ? __ldg(p.slot_mapping + i)
                                                 : __ldg(p.x_slots + (i - p.num_tokens));
             if (sl >= 0 && sl < p.num_slots)
@@ -797,9 +803,9 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
         const int n4 = static_cast<int>(crossing_set_bytes(p.num_slots, p.x_tokens) >> 4);
         const uint32_t f = bitmap ? 0u : kEmptySlot;
         const uint4 fill = make_uint4(f, f, f, f);
-        for (int i = threadIdx.x; i < n4; i += kKvThreads) tab4[i] = fill;
+        for (int i = threadIdx.x; i < n4; i += kThreads) tab4[i] = fill;
         __syncthreads();
-        for (int64_t i = threadIdx.x; i < p.x_tokens; i += kKvThreads) {
+        for (int64_t i = threadIdx.x; i < p.x_tokens; i += kThreads) {
             const int64_t sl = __ldg(p.x_slots + i);
             if (sl >= 0 && sl < p.num_slots) {
                 const uint32_t key = static_cast<uint32_t>(sl);
@@ -847,7 +853,7 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
     }
 
     if (kAmax) {
-        __shared__ uint32_t red[2][kKvWarps];
+        __shared__ uint32_t red[2][kWarps];
         uint32_t km = __reduce_max_sync(0xFFFFFFFFu, absmax_bits16(kacc));
         uint32_t vm = __reduce_max_sync(0xFFFFFFFFu, absmax_bits16(vacc));
         const int w = threadIdx.x >> 5;
@@ -858,7 +864,7 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_pass_kernel(const KvPass p) 
         __syncthreads();
         if (threadIdx.x == 0) {
 #pragma unroll
-            for (int i = 1; i < kKvWarps; ++i) {
+            for (int i = 1; i < kWarps; ++i) {
                 km = max(km, red[0][i]);
                 vm = max(vm, red[1][i]);
             }
@@ -1030,18 +1036,21 @@ cudaError_t launch(void (*kernel)(Params...), int grid, int block, size_t smem,
 
 template <bool A, bool S, bool W, bool X>
 cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
-    auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, X, 64> : kv_pass_kernel<A, S, W, X, 0>;
+    constexpr int kThreads = X ? 512 : kKvThreads;
+    constexpr int kWarps = kThreads / 32;
+    auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, X, 64, kThreads>
+                                 : kv_pass_kernel<A, S, W, X, 0, kThreads>;
     const int64_t tokens = p.num_tokens + (X ? p.x_tokens : 0);
-    const int64_t per_cta = (W && !A && !S && !X) ? 2 * kKvWarps : kKvWarps;   // see kTwo
+    const int64_t per_cta = (W && !A && !S && !X) ? 2 * kWarps : kWarps;   // see kTwo
     const int64_t wanted = (tokens + per_cta - 1) / per_cta;
     const size_t smem =
         !X ? 0
            : p.last_writer ? (size_t{8} << last_writer_log2(tokens))
                            : static_cast<size_t>(crossing_set_bytes(p.num_slots, p.x_tokens));
     int grid = 1;
-    cudaError_t e = grid_for(kernel, kKvThreads, smem, wanted, &grid);
+    cudaError_t e = grid_for(kernel, kThreads, smem, wanted, &grid);
     if (e != cudaSuccess) return e;
-    return launch(kernel, grid, kKvThreads, smem, stream, p);
+    return launch(kernel, grid, kThreads, smem, stream, p);
 }
 
 }  // namespace
