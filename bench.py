@@ -662,11 +662,37 @@ def measured_peaks() -> dict:
         return {"hbm_gbs": 6650.0, "source": "fallback 6.65 TB/s"}
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and whitespace (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            if not c.isspace():
+                out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def source_hash() -> str:
+    """Hash of the kernel sources' code (comments and whitespace ignored), the
+    key under which ncu figures are recorded in profiles/traffic.json."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_group_b200", "csrc", "*"))):
-        with open(p, "rb") as fh:
-            h.update(fh.read())
+        with open(p, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -428,16 +428,17 @@ group_quant_kmajor_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
 // ---------------------------------------------------------------------------
 // 2./3. KV pass: absmax, staging copy and quantize-and-scatter
 //
-// One warp per token (grid-stride).  Lane l owns 16-byte chunks l and l+32 of
-// the K row and of the V row, so every load and store instruction of the warp
-// is one contiguous run (512 B of bf16 in, 256 B of codes out).  The slot
-// decides where the codes land: one token's entry is E contiguous bytes of the
-// pool, written as 32 8-byte stores per instruction.
+// One warp per token (grid-stride; the plain write takes two tokens per warp
+// on half the grid).  Lane l owns 16-byte chunks l and l+32 of the K row and
+// of the V row, so every load and store instruction of the warp is one
+// contiguous run (512 B of bf16 in, 256 B of codes out).  The slot decides
+// where the codes land: one token's entry is E contiguous bytes of the pool,
+// written as 32 8-byte stores per instruction.
 //
-// Each warp issues its first token's loads before anything else.  The scales
-// (a dependent load, and for a freeze an IEEE division and a reciprocal) are
-// resolved once per CTA by thread 0 while those loads are in flight, and
-// shared through shared memory.
+// Each warp issues its first token's loads before anything else, then
+// resolves the scales itself (a dependent 8-byte load; for a freeze the frozen
+// scale from the device maxima) while those loads are in flight.  CTAs are 256
+// threads, 512 for the merged freeze launch (see kv_pass_kernel).
 
 constexpr int kKvThreads = 256;
 constexpr int kKvWarps = kKvThreads / 32;
