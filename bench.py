@@ -26,7 +26,6 @@ the step issues them (one per layer, back to back), timed the same way.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -686,12 +685,16 @@ def _code_only(text: str) -> str:
     return "".join(out)
 
 
+KERNEL_SOURCES = ("fp8q_kernels.cu", "fp8q_internal.h")   # device code and launch geometry
+
+
 def source_hash() -> str:
-    """Hash of the kernel sources' code (comments and whitespace ignored), the
-    key under which ncu figures are recorded in profiles/traffic.json."""
+    """Hash of the kernels' code (comments and whitespace ignored), the key
+    under which ncu figures are recorded in profiles/traffic.json."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_group_b200", "csrc", "*"))):
-        with open(p, encoding="utf-8") as fh:
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_group_b200", "csrc", name),
+                  encoding="utf-8") as fh:
             h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 

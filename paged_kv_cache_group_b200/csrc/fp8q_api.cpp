@@ -24,7 +24,7 @@ namespace {
 
 using fp8q::KvPass;
 
-constexpr int32_t kVersion = 10000;  // 1.0.0
+constexpr int32_t kVersion = 10100;  // 1.1.0: fp8_group_quant_kmajor, fp8_kv_calib_restore
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

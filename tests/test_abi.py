@@ -32,7 +32,7 @@ def test_every_declared_function_is_exported_and_bound():
 
 
 def test_version_and_status_strings():
-    assert fp8q.version() == 10000
+    assert fp8q.version() == 10100
     assert fp8q.lib.fp8q_status_string(0) == b"ok"
     assert fp8q.lib.fp8q_status_string(-1) == b"invalid argument"
     assert fp8q.lib.fp8q_status_string(-3) == b"calibration call out of order"
