@@ -335,6 +335,16 @@ def fp8_kv_calib_window_noalloc(k: torch.Tensor, v: torch.Tensor, slot_mapping: 
         _ptr(scales_out), _stream(stream)))
 
 
+def allreduce_kv_maxima(calibrator, group=None) -> None:
+    """KV heads sharded over ranks, one scale for all of them: after
+    ``observe()`` returns STEP_FREEZE for the batch that reaches the window and
+    before ``freeze_replay()``, make every rank's device |K| and |V| maxima the
+    maximum over the group (one all-reduce of two fp32 values, enqueued on the
+    current stream).  Every rank then freezes the same scales."""
+    import torch.distributed as dist
+    dist.all_reduce(calibrator.state[0:2], op=dist.ReduceOp.MAX, group=group)
+
+
 def save_scales(calibrators, path: str) -> None:
     """Write every layer's frozen scales to a JSON file (exact hex floats)."""
     import json

@@ -1,5 +1,6 @@
-"""Host-side logic of bench.py on CPU: the multi-rank aggregation (gloo,
-world size 2) and the reference arm's JSON contract."""
+"""Host-side logic on CPU: bench.py's multi-rank aggregation (gloo, world
+size 2) and its reference arm's JSON contract, and the all-reduce of the KV
+maxima for heads sharded over ranks (gloo, world size 2)."""
 import argparse
 import os
 import socket
@@ -86,3 +87,34 @@ def test_algorithmic_bytes():
 def test_cli_rejects_short_warmup():
     with pytest.raises(SystemExit):
         bench.parse_args(["--warmup", "2"])
+
+
+def _maxima_rank(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import types
+    import torch.distributed as dist
+    import paged_kv_cache_group_b200 as fp8q
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # a calibrator's state layout {k_amax, v_amax, k_scale, v_scale} on the host
+    cal = types.SimpleNamespace(state=torch.tensor([1.5 + rank, 7.0 - 3 * rank, 2.0, 2.0]))
+    fp8q.allreduce_kv_maxima(cal)
+    out[rank] = cal.state.tolist()
+    dist.destroy_process_group()
+
+
+def test_sharded_heads_share_the_maxima_before_the_freeze():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_maxima_rank, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0
+        res = dict(out)
+    # maxima reduced, scales untouched
+    assert res[0] == res[1] == [2.5, 7.0, 2.0, 2.0]
