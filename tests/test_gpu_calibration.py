@@ -313,3 +313,36 @@ def test_saved_scales_restore_a_frozen_calibrator(tmp_path):
         g.cal.restore(ks, vs)
     assert ei.value.status == -3
     fresh.cal.close()
+
+
+def test_unfused_freeze_with_the_maxima_allreduce_on_one_rank():
+    """observe -> allreduce_kv_maxima (NCCL, one rank) -> freeze_replay, on the
+    device state: the pools equal the oracle's, as without the all-reduce."""
+    import socket
+    import torch.distributed as dist
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        spec, batches, _ = workloads.calib_window()
+        g = GpuLayer(spec, workloads.CALIB_WINDOW, 1.0, fused=False)
+        c, kp, vp = _oracle_layer(spec, workloads.CALIB_WINDOW, 1.0)
+        for b in batches:
+            k, v = _rows(b.k, spec.heads, spec.dim), _rows(b.v, spec.heads, spec.dim)
+            slots = dev(b.slot_mapping)
+            step = g.cal.observe(k, v, slots)
+            if step == fp8q.STEP_FREEZE:
+                fp8q.allreduce_kv_maxima(g.cal)
+                g.cal.freeze_replay(g.kp4, g.vp4)
+            fp8q.fp8_kv_write(k, v, slots, g.kp4, g.vp4, scale_dev=g.cal.scale_dev)
+            cal.run_calibrated_writes(c, [cal.KvBatch(b.k, b.v, b.slot_mapping, b.key_stride,
+                                                      b.value_stride)],
+                                      spec.heads, spec.dim, kp, vp, spec.block_size,
+                                      spec.cache_stride, spec.num_blocks)
+        gk, gv = host(g.kp), host(g.vp)
+        assert np.array_equal(gk, kp), first_mismatch(gk, kp)
+        assert np.array_equal(gv, vp), first_mismatch(gv, vp)
+        _assert_frozen_state(g, c)
+    finally:
+        dist.destroy_process_group()
