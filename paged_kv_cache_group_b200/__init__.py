@@ -61,6 +61,36 @@ def _bf16_rows(t: torch.Tensor, name: str):
     return rows, (t.stride(0) if rows > 1 else inner), inner
 
 
+def _kv_rows(k: torch.Tensor, v: torch.Tensor):
+    """K and V ``[T, heads, dim]`` of the same shape (rows contiguous, row
+    strides may differ); returns (T, key_stride, value_stride, heads, dim).
+    The shapes are checked before anything else, so a mismatched V is refused
+    whatever device it is on."""
+    if k.dim() != 3 or v.dim() != 3:
+        raise ValueError("k and v must both be [T, heads, dim]")
+    if tuple(k.shape) != tuple(v.shape):
+        raise ValueError(f"k and v must have the same shape, got {tuple(k.shape)} and "
+                         f"{tuple(v.shape)}")
+    t, ks, _ = _bf16_rows(k, "k")
+    _, vs, _ = _bf16_rows(v, "v")
+    return t, ks, vs, k.shape[1], k.shape[2]
+
+
+def _check_slots(slot_mapping: torch.Tensor, t: int) -> None:
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() < t:
+        raise ValueError("slot_mapping must be int64 with one entry per token")
+    if t and (not slot_mapping.is_cuda or not slot_mapping.is_contiguous()):
+        raise ValueError("slot_mapping must be a contiguous CUDA tensor")
+
+
+def _check_scale_pair(t: torch.Tensor | None, name: str) -> None:
+    """A device ``{k, v}`` fp32 pair the library reads or writes."""
+    if t is None:
+        return
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.numel() < 2:
+        raise ValueError(f"{name} must be a contiguous CUDA float32 tensor of 2 elements")
+
+
 # ---------------------------------------------------------------------------
 # activation quantization
 
@@ -140,14 +170,10 @@ def fp8_kv_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
     """reshape_and_cache_fp8: K, V ``[T, heads, dim]`` bf16 into the pools at
     ``slot_mapping`` (int64, -1 skips), per-tensor scales by value or from the
     device ``scale_dev [2]``."""
-    t, ks, e = _bf16_rows(k, "k")
-    t2, vs, e2 = _bf16_rows(v, "v")
-    if (t, e) != (t2, e2) or k.dim() != 3:
-        raise ValueError("k and v must both be [T, heads, dim]")
-    heads, dim = k.shape[1], k.shape[2]
-    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() < t:
-        raise ValueError("slot_mapping must be int64 with one entry per token")
-    nb, bs, cs = _pool_geometry(k_pool, v_pool, e)
+    t, ks, vs, heads, dim = _kv_rows(k, v)
+    _check_slots(slot_mapping, t)
+    _check_scale_pair(scale_dev, "scale_dev")
+    nb, bs, cs = _pool_geometry(k_pool, v_pool, heads * dim)
     _check("fp8_kv_write", lib.fp8_kv_write(
         _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, heads, dim, _ptr(k_pool),
         _ptr(v_pool), bs, cs, nb, float(k_scale), float(v_scale), _ptr(scale_dev),
@@ -167,19 +193,19 @@ def fp8_kv_write_layers(ks, vs, slot_mappings, k_pools, v_pools, k_scales=None, 
         raise ValueError(f"at most {_abi.MAX_LAYERS} layers per launch")
     if n == 0:
         return
-    t, kst, e = _bf16_rows(ks[0], "k")
-    _, vst, _ = _bf16_rows(vs[0], "v")
-    heads, dim = ks[0].shape[1], ks[0].shape[2]
+    t, kst, vst, heads, dim = _kv_rows(ks[0], vs[0])
+    e = heads * dim
     nb, bs, cs = _pool_geometry(k_pools[0], v_pools[0], e)
     arr = (_abi.KvLayer * n)()
     for i in range(n):
-        ti, ksi, _ = _bf16_rows(ks[i], "k")
-        _, vsi, _ = _bf16_rows(vs[i], "v")
-        if (ti, ksi, vsi) != (t, kst, vst) or tuple(ks[i].shape[1:]) != (heads, dim):
+        ti, ksi, vsi, hi, di = _kv_rows(ks[i], vs[i])
+        if (ti, ksi, vsi, hi, di) != (t, kst, vst, heads, dim):
             raise ValueError("all layers must share the row shape and strides")
+        _check_slots(slot_mappings[i], t)
         if _pool_geometry(k_pools[i], v_pools[i], e) != (nb, bs, cs):
             raise ValueError("all layers' pools must share one geometry")
         sd = None if scale_devs is None else scale_devs[i]
+        _check_scale_pair(sd, "scale_devs[i]")
         arr[i] = _abi.KvLayer(_ptr(ks[i]), _ptr(vs[i]), _ptr(slot_mappings[i]), _ptr(k_pools[i]),
                               _ptr(v_pools[i]), _ptr(sd),
                               float(k_scales[i]) if k_scales is not None else 1.0,
@@ -190,12 +216,10 @@ def fp8_kv_write_layers(ks, vs, slot_mappings, k_pools, v_pools, k_scales=None, 
 
 def fp8_kv_amax_observe(k: torch.Tensor, v: torch.Tensor, amax_dev: torch.Tensor, stream=None):
     """Max-accumulate max|K| and max|V| into the device fp32 ``amax_dev [2]``."""
-    t, ks, e = _bf16_rows(k, "k")
-    _, vs, _ = _bf16_rows(v, "v")
-    if amax_dev.dtype != torch.float32 or amax_dev.numel() < 2:
-        raise ValueError("amax_dev must be a float32 tensor of 2 elements")
+    t, ks, vs, heads, dim = _kv_rows(k, v)
+    _check_scale_pair(amax_dev, "amax_dev")
     _check("fp8_kv_amax_observe", lib.fp8_kv_amax_observe(
-        _ptr(k), _ptr(v), ks, vs, t, k.shape[1], k.shape[2], _ptr(amax_dev), _stream(stream)))
+        _ptr(k), _ptr(v), ks, vs, t, heads, dim, _ptr(amax_dev), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------
@@ -259,12 +283,12 @@ class KvCalibration:
 
     def observe(self, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
                 stream=None) -> int:
-        t, ks, e = _bf16_rows(k, "k")
-        _, vs, _ = _bf16_rows(v, "v")
+        t, ks, vs, heads, dim = _kv_rows(k, v)
+        _check_slots(slot_mapping, t)
         step = ctypes.c_int32()
         _check("fp8_kv_calib_observe", lib.fp8_kv_calib_observe(
-            self.handle, _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, k.shape[1],
-            k.shape[2], _stream(stream), ctypes.byref(step)))
+            self.handle, _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, heads, dim,
+            _stream(stream), ctypes.byref(step)))
         return step.value
 
     def freeze_replay(self, k_pool: torch.Tensor, v_pool: torch.Tensor, stream=None) -> int:
@@ -277,14 +301,13 @@ class KvCalibration:
 
     def observe_write(self, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
                       k_pool: torch.Tensor, v_pool: torch.Tensor, stream=None) -> int:
-        t, ks, e = _bf16_rows(k, "k")
-        _, vs, _ = _bf16_rows(v, "v")
-        nb, bs, cs = _pool_geometry(k_pool, v_pool, e)
+        t, ks, vs, heads, dim = _kv_rows(k, v)
+        _check_slots(slot_mapping, t)
+        nb, bs, cs = _pool_geometry(k_pool, v_pool, heads * dim)
         step = ctypes.c_int32()
         _check("fp8_kv_calib_observe_write", lib.fp8_kv_calib_observe_write(
-            self.handle, _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, k.shape[1],
-            k.shape[2], _ptr(k_pool), _ptr(v_pool), bs, cs, nb, _stream(stream),
-            ctypes.byref(step)))
+            self.handle, _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), t, heads, dim,
+            _ptr(k_pool), _ptr(v_pool), bs, cs, nb, _stream(stream), ctypes.byref(step)))
         return step.value
 
     def restore(self, k_scale: float, v_scale: float, stream=None) -> None:
@@ -320,29 +343,34 @@ def fp8_kv_calib_window_noalloc(k: torch.Tensor, v: torch.Tensor, slot_mapping: 
     the caller or the library's user: the scratch is a fixed array inside the
     library (see include/fp8q.h).  ``k``/``v`` hold every batch's rows back to
     back; ``batch_tokens`` lists each batch's token count."""
-    t, ks, e = _bf16_rows(k, "k")
-    _, vs, _ = _bf16_rows(v, "v")
+    t, ks, vs, heads, dim = _kv_rows(k, v)
     counts = [int(n) for n in batch_tokens]
     if sum(counts) != t:
         raise ValueError("batch_tokens must add up to the rows of k and v")
-    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() < t:
-        raise ValueError("slot_mapping must be int64 with one entry per token")
-    nb, bs, cs = _pool_geometry(k_pool, v_pool, e)
+    _check_slots(slot_mapping, t)
+    _check_scale_pair(scales_out, "scales_out")
+    nb, bs, cs = _pool_geometry(k_pool, v_pool, heads * dim)
     arr = (ctypes.c_int64 * max(len(counts), 1))(*counts)
     _check("fp8_kv_calib_window_noalloc", lib.fp8_kv_calib_window_noalloc(
-        _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), arr, len(counts), k.shape[1], k.shape[2],
+        _ptr(k), _ptr(v), ks, vs, _ptr(slot_mapping), arr, len(counts), heads, dim,
         int(window_tokens), float(headroom), _ptr(k_pool), _ptr(v_pool), bs, cs, nb,
         _ptr(scales_out), _stream(stream)))
 
 
-def allreduce_kv_maxima(calibrator, group=None) -> None:
+def allreduce_kv_maxima(calibrator, group=None, stream=None) -> None:
     """KV heads sharded over ranks, one scale for all of them: after
     ``observe()`` returns STEP_FREEZE for the batch that reaches the window and
     before ``freeze_replay()``, make every rank's device |K| and |V| maxima the
-    maximum over the group (one all-reduce of two fp32 values, enqueued on the
-    current stream).  Every rank then freezes the same scales."""
+    maximum over the group (one all-reduce of two fp32 values).  Every rank
+    then freezes the same scales.  Pass the ``stream`` that ``observe()`` and
+    ``freeze_replay()`` use (default: the current stream): the all-reduce is
+    ordered after that stream's absmax kernels and before its replay."""
     import torch.distributed as dist
-    dist.all_reduce(calibrator.state[0:2], op=dist.ReduceOp.MAX, group=group)
+    if stream is None or isinstance(stream, int):
+        dist.all_reduce(calibrator.state[0:2], op=dist.ReduceOp.MAX, group=group)
+        return
+    with torch.cuda.stream(stream):
+        dist.all_reduce(calibrator.state[0:2], op=dist.ReduceOp.MAX, group=group)
 
 
 def save_scales(calibrators, path: str) -> None:
