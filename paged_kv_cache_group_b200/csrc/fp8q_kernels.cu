@@ -13,18 +13,21 @@
 // By Markstein's theorem (r within half an ulp of 1/s, q0 within one ulp of
 // x/s, no underflow or overflow) q is the correctly rounded x/s.  The three
 // steps run on pairs of values (fma.rn.f32x2, two independent IEEE
-// operations per instruction).  This form can turn the quotient of x = -0
-// into +0, so after the conversion the sign bit of every code whose input is
-// negative is set again from the bf16 sign bits (a no-op for every other
-// negative input, whose code already carries it).  When s is a power of two,
-// r = 1/s exactly and RN(x * r) is already the quotient: one product.  For
-// the activation quantizer this was checked exhaustively over every pair of
-// bf16 x and bf16 group maximum; for a per-tensor scale the reciprocal form
-// is used only while the scale lies in [2^-64, 2^64] (x clamped so that x * r
-// cannot overflow, which only changes values that saturate anyway), and
-// __fdiv_rn is used outside that range.  The quotient is then rounded by the
-// hardware conversion cvt.rn.satfinite.e4m3x2.f32: nearest-even, saturating
-// to +-448.
+// operations per instruction).  The residual step is rounded toward -inf: a
+// nonzero residual is exact, so the mode changes nothing but the sign of an
+// exact zero, and with it x = -0 (and a negative x whose quotient underflows)
+// keeps its sign through q = q0 + e*r, as IEEE division does.  When s is a
+// power of two, r = 1/s exactly and RN(x * r) is already the quotient: one
+// product.  A per-tensor scale may be small enough that x * r overflows for
+// huge x, so there the product uses r' = r * 2^-k in [0.5, 1) (and s' =
+// s * 2^k) and is scaled back by an exact multiply by 2^k before the
+// correction; a product that overflows there is infinite and saturates to
+// +-448, the code of the (equally huge) quotient.  Both forms were checked
+// on the CPU against IEEE division: the group form over every pair of bf16 x
+// and bf16 group maximum, the per-tensor form over every bf16 x at 2400
+// scales in [2^-64, 2^64]; codes agree everywhere.  Scales outside that
+// range use __fdiv_rn.  The quotient is then rounded by the hardware
+// conversion cvt.rn.satfinite.e4m3x2.f32: nearest-even, saturating to +-448.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -108,13 +111,6 @@ __device__ __forceinline__ uint32_t absmax_bits16(uint32_t acc) {
     return max(acc & 0xFFFFu, acc >> 16);
 }
 
-__device__ __forceinline__ uint32_t clamp_bf16x2(uint32_t w, uint32_t lo2, uint32_t hi2) {
-    uint32_t d;
-    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(w), "r"(lo2));
-    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(d), "r"(hi2));
-    return d;
-}
-
 // Two fp32 values to two E4M3 codes: byte 0 <- lo, byte 1 <- hi.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     unsigned short d;
@@ -159,19 +155,24 @@ __device__ __forceinline__ PairDivisor pair_divisor(const Divisor &d) {
     return PairDivisor{pair(d.r, d.r), pair(-d.s, -d.s)};
 }
 
-// Correctly rounded quotients of a pair (see the file comment).
+__device__ __forceinline__ uint64_t fma2_rm(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Correctly rounded quotients of a pair, signs of zero included (see the
+// file comment).
 __device__ __forceinline__ uint64_t quotient2(uint64_t x, const PairDivisor &d) {
     const uint64_t q0 = mul2(x, d.r2);
-    const uint64_t e = fma2(q0, d.ns2, x);
+    const uint64_t e = fma2_rm(q0, d.ns2, x);
     return fma2(e, d.r2, q0);
 }
 
-// Codes of four values (bf16x2 words w0, w1) with the sign of every negative
-// input's code set from the bf16 sign bits.
+// Codes of four values (bf16x2 words w0, w1).
 __device__ __forceinline__ uint32_t encode4(uint32_t w0, uint32_t w1, const PairDivisor &d) {
-    const uint32_t c = e4m3x2_pair(quotient2(pair_of_bf16x2(w0), d)) |
-                       (e4m3x2_pair(quotient2(pair_of_bf16x2(w1), d)) << 16);
-    return c | (__byte_perm(w0, w1, 0x7531) & 0x80808080u);
+    return e4m3x2_pair(quotient2(pair_of_bf16x2(w0), d)) |
+           (e4m3x2_pair(quotient2(pair_of_bf16x2(w1), d)) << 16);
 }
 
 // Codes of four values for a power-of-two scale: r is exact, one product.
@@ -210,65 +211,86 @@ __device__ __forceinline__ uint2 encode8_div(const uint4 &w, float s) {
     return o;
 }
 
-// Per-tensor encoder.  Fast path: the reciprocal form, with x first clamped
-// to +-T when r > 1 so that x * r cannot overflow (T = s * 1024 rounded up to
-// bf16: any |x| >= T saturates anyway, and T * r stays far from overflow;
-// with r <= 1 no bf16 value can overflow).  Scales outside [2^-64, 2^64]:
-// IEEE division per element.
+// Per-tensor quotients of a pair with the product taken on r' = r * 2^-k and
+// scaled back by c = 2^k (see the file comment): no overflow before the
+// correction, an infinite result only where the quotient itself is huge.
+struct ScaledDivisor {
+    uint64_t rs2;    // {r', r'}
+    uint64_t nss2;   // {-s', -s'}
+    uint64_t c2;     // {2^k, 2^k}
+    uint64_t r2;     // {r, r}
+};
+
+__device__ __forceinline__ uint64_t quotient2_scaled(uint64_t x, const ScaledDivisor &d) {
+    const uint64_t q0 = mul2(x, d.rs2);
+    const uint64_t e = fma2_rm(q0, d.nss2, x);
+    return fma2(e, d.r2, mul2(q0, d.c2));
+}
+
+__device__ __forceinline__ uint2 encode8_scaled(const uint4 &w, const ScaledDivisor &d) {
+    uint2 o;
+    o.x = e4m3x2_pair(quotient2_scaled(pair_of_bf16x2(w.x), d)) |
+          (e4m3x2_pair(quotient2_scaled(pair_of_bf16x2(w.y), d)) << 16);
+    o.y = e4m3x2_pair(quotient2_scaled(pair_of_bf16x2(w.z), d)) |
+          (e4m3x2_pair(quotient2_scaled(pair_of_bf16x2(w.w), d)) << 16);
+    return o;
+}
+
+// Per-tensor encoder.  Scales in [2^-64, 2^64]: the reciprocal form, plain
+// when r < 1 (no bf16 value can overflow x * r) and scaled otherwise; a
+// power-of-two scale takes one product.  Other scales: IEEE division per
+// element.
 struct TensorEncoder {
-    Divisor d;
-    uint32_t lo2, hi2;   // clamp bounds as bf16x2 (-T, T)
+    float s;
+    PairDivisor pd;      // {r, r}, {-s, -s}
+    ScaledDivisor sd;
     bool fast;
     bool pow2;           // s is a power of two: RN(x * r) is the quotient
-    bool clamp;
+    bool scaled;         // r >= 1: take the product on r' and scale back
     bool ok;             // scale is a positive number
 
-    __device__ __forceinline__ void init(float s) {
+    __device__ __forceinline__ void init(float scale) {
+        s = scale;
         ok = s > 0.0f;   // false for NaN
         fast = (s >= 0x1p-64f) && (s <= 0x1p64f);
         pow2 = fast && (__float_as_uint(s) & 0x7FFFFFu) == 0;
-        d.s = s;
-        d.r = __frcp_rn(s);
-        clamp = d.r > 1.0f;
-        uint32_t u = __float_as_uint(__fmul_rn(s, 1024.0f));
-        if (u & 0xFFFFu) u += 0x10000u;
-        const uint32_t t = (u >> 16) & 0x7FFFu;
-        hi2 = t | (t << 16);
-        lo2 = hi2 | 0x80008000u;
+        const float r = __frcp_rn(s);
+        pd.r2 = pair(r, r);
+        pd.ns2 = pair(-s, -s);
+        // r' = r * 2^-k in [0.5, 1), s' = s * 2^k, c = 2^k: exponent-field
+        // arithmetic, exact for the normal r and s of the fast range
+        const int k = r >= 1.0f ? static_cast<int>((__float_as_uint(r) >> 23) & 0xFF) - 126 : 0;
+        scaled = k > 0;
+        const float rs = __uint_as_float(__float_as_uint(r) - (static_cast<uint32_t>(k) << 23));
+        const float ss = __uint_as_float(__float_as_uint(s) + (static_cast<uint32_t>(k) << 23));
+        const float c = __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
+        sd.rs2 = pair(rs, rs);
+        sd.nss2 = pair(-ss, -ss);
+        sd.c2 = pair(c, c);
+        sd.r2 = pd.r2;
     }
 
-    __device__ __forceinline__ static uint4 clamp4(uint4 w, uint32_t lo2, uint32_t hi2) {
-        w.x = clamp_bf16x2(w.x, lo2, hi2);
-        w.y = clamp_bf16x2(w.y, lo2, hi2);
-        w.z = clamp_bf16x2(w.z, lo2, hi2);
-        w.w = clamp_bf16x2(w.w, lo2, hi2);
-        return w;
-    }
+    // The caller knows |x| / s <= 448 for every x it encodes (the maxima the
+    // scale comes from cover them): x * r cannot overflow, so the plain form.
+    __device__ __forceinline__ void within_range() { scaled = false; }
 
-    // Two chunks of a row.  Power-of-two scale: one product per value (an
-    // overflow to infinity saturates like the quotient it stands for).
-    // Otherwise only magnitudes at or beyond T can overflow x * r, and T is
-    // far above any realistic K/V, so the clamp runs only when the pair's
-    // largest magnitude reaches it.
-    __device__ __forceinline__ void encode2(uint4 a, uint4 b, uint2 &oa, uint2 &ob) const {
+    // Two chunks of a row.
+    __device__ __forceinline__ void encode2(const uint4 &a, const uint4 &b, uint2 &oa,
+                                            uint2 &ob) const {
         if (pow2) {
-            const uint64_t r2 = pair(d.r, d.r);
-            oa = encode8_pow2(a, r2);
-            ob = encode8_pow2(b, r2);
+            oa = encode8_pow2(a, pd.r2);
+            ob = encode8_pow2(b, pd.r2);
         } else if (fast) {
-            if (clamp) {
-                const uint32_t m = absmax_bits16(absmax_uint4(absmax_uint4(0u, a), b));
-                if (m >= (hi2 & 0xFFFFu)) {
-                    a = clamp4(a, lo2, hi2);
-                    b = clamp4(b, lo2, hi2);
-                }
+            if (scaled) {
+                oa = encode8_scaled(a, sd);
+                ob = encode8_scaled(b, sd);
+            } else {
+                oa = encode8(a, pd);
+                ob = encode8(b, pd);
             }
-            const PairDivisor pd = pair_divisor(d);
-            oa = encode8(a, pd);
-            ob = encode8(b, pd);
         } else {
-            oa = encode8_div(a, d.s);
-            ob = encode8_div(b, d.s);
+            oa = encode8_div(a, s);
+            ob = encode8_div(b, s);
         }
     }
 };
@@ -571,9 +593,9 @@ __device__ __forceinline__ void resolve_scales(const KvPass &p, TensorEncoder &k
     if (p.freeze_amax != nullptr) {
         // Every row a freeze pass writes (staged or crossing) went into the
         // maxima the scale comes from, so |x| / s <= 448 / headroom <= 448 and
-        // x * r cannot overflow: the clamp is never needed.
-        kenc.clamp = false;
-        venc.clamp = false;
+        // x * r cannot overflow.
+        kenc.within_range();
+        venc.within_range();
     }
     if (!(kenc.ok && venc.ok) && blockIdx.x == 0 && threadIdx.x == 0)
         atomicOr(&g_error_word, kErrScale);
