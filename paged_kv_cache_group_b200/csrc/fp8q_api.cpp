@@ -69,11 +69,6 @@ bool valid_pools(const void *k_pool, const void *v_pool, int32_t block_size,
 // ---------------------------------------------------------------------------
 // calibrator
 
-struct StagedBatch {
-    int64_t offset_tokens;
-    int64_t num_tokens;
-};
-
 enum CalibPhase : int32_t { kCalibrating = 0, kFreezePending = 1, kFrozen = 2 };
 
 struct fp8_kv_calib {
@@ -97,7 +92,8 @@ struct fp8_kv_calib {
     int64_t freeze_tokens = 0;
     int64_t replayed_tokens = 0;
     int64_t replayed_batches = 0;
-    std::vector<StagedBatch> batches;
+    // rows of each staged batch, in arrival order (packed in staging)
+    std::vector<int64_t> staged_counts;
 };
 
 namespace {
@@ -144,7 +140,7 @@ fp8q_status plan_observe(fp8_kv_calib *c, const void *k, const void *v, int64_t 
         pass->stage_v = c->stage_v;
         pass->stage_slots = c->stage_slots;
         pass->stage_offset = c->used_tokens;
-        c->batches.push_back({c->used_tokens, num_tokens});
+        c->staged_counts.push_back(num_tokens);
         c->used_tokens += num_tokens;
         *step = FP8Q_STEP_STAGE;
     } else {
@@ -154,13 +150,11 @@ fp8q_status plan_observe(fp8_kv_calib *c, const void *k, const void *v, int64_t 
     return FP8Q_OK;
 }
 
-// The freeze's device work: every staged batch is rewritten, in the order it
-// was staged, at the scales frozen from the device maxima; the first launch
-// also publishes those scales to state_dev.  When `crossing` is given (the
-// batch that reached the window, as a write pass reading the published
-// scales) and fits in one launch with the last staged batch, the two share a
-// launch; otherwise the crossing batch is written by its own launch after the
-// replay.  Either way each slot ends with its last writer in arrival order.
+// The freeze's device work (fp8q::enqueue_freeze_replay): every staged batch
+// rewritten, in arrival order, at the scales frozen from the device maxima,
+// the scales published to state_dev, then `crossing` (the batch that reached
+// the window, as a write pass reading the published scales) if given.  Each
+// slot ends with its last writer in arrival order.
 fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t block_size,
                        int64_t cache_stride, int64_t num_blocks, cudaStream_t stream,
                        int64_t *replayed, const KvPass *crossing, bool chained = false) {
@@ -170,8 +164,6 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
     KvPass p;
     p.do_write = true;
     p.elems = static_cast<int32_t>(c->elems);
-    p.key_stride = c->elems;       // staging rows are packed
-    p.value_stride = c->elems;
     p.k_pool = static_cast<uint8_t *>(k_pool);
     p.v_pool = static_cast<uint8_t *>(v_pool);
     p.block_size = block_size;
@@ -181,90 +173,17 @@ fp8q_status run_replay(fp8_kv_calib *c, void *k_pool, void *v_pool, int32_t bloc
     p.freeze_amax = amax_bits(c);
     p.headroom = c->headroom;
     p.scale_out = scale_dev(c);
-    // chained: the previous launch on the stream is this call's own amax pass,
-    // and every launch below follows one of these; the staged rows and the
-    // crossing batch were all written before that amax pass was enqueued.
-    p.early_loads = chained;
-
-    // Last staged batch with rows: the one the crossing batch joins.
-    int64_t last = -1;
-    for (int64_t i = 0; i < static_cast<int64_t>(c->batches.size()); ++i)
-        if (c->batches[i].num_tokens > 0) last = i;
-    KvPass probe = p;
-    if (crossing != nullptr) {
-        probe.x_tokens = crossing->num_tokens;
-    }
-    const bool merge = crossing != nullptr && crossing->num_tokens > 0 &&
-                       crossing->elems == p.elems && fp8q::can_merge_crossing(probe);
-    auto with_crossing = [&](KvPass q) {
-        q.xk = crossing->k;
-        q.xv = crossing->v;
-        q.x_key_stride = crossing->key_stride;
-        q.x_value_stride = crossing->value_stride;
-        q.x_slots = crossing->slot_mapping;
-        q.x_tokens = crossing->num_tokens;
-        return q;
-    };
-
     int64_t rewritten = 0;
-    bool published = false;
-
-    // Two or more staged batches with rows: every staged row and the crossing
-    // batch in one launch, each slot written by its last writer in arrival
-    // order, when the window is small enough for the last-writer table.
-    int64_t with_rows = 0;
-    for (const StagedBatch &b : c->batches) with_rows += b.num_tokens > 0;
-    const int64_t whole_rows = c->used_tokens + (merge ? crossing->num_tokens : 0);
-    if (with_rows >= 2 && whole_rows <= fp8q::kMaxLastWriterTokens &&
-        p.num_slots <= 0x7FFFFFFF) {
-        KvPass q = merge ? with_crossing(p) : p;
-        q.k = c->stage_k;
-        q.v = c->stage_v;
-        q.slot_mapping = c->stage_slots;
-        q.num_tokens = c->used_tokens;
-        q.last_writer = true;
-        if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
-        rewritten = c->used_tokens;
-        published = true;
-        if (crossing != nullptr && !merge) {
-            KvPass x = *crossing;
-            x.early_loads = chained;
-            if (fp8q::launch_kv_pass(x, stream) != cudaSuccess) return FP8Q_ECUDA;
-        }
-    } else if (merge && last < 0) {
-        // nothing staged with rows: the crossing batch alone, publishing the scales
-        KvPass q = with_crossing(p);
-        q.num_tokens = 0;
-        if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
-        published = true;
-    } else {
-        for (int64_t i = 0; i < static_cast<int64_t>(c->batches.size()); ++i) {
-            const StagedBatch &b = c->batches[i];
-            if (b.num_tokens == 0 && published) continue;
-            p.k = c->stage_k + b.offset_tokens * c->elems;
-            p.v = c->stage_v + b.offset_tokens * c->elems;
-            p.slot_mapping = c->stage_slots + b.offset_tokens;
-            p.num_tokens = b.num_tokens;
-            const KvPass q = (merge && i == last) ? with_crossing(p) : p;
-            if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
-            rewritten += b.num_tokens;
-            published = true;
-        }
-        if (!published) {
-            p.num_tokens = 0;
-            if (fp8q::launch_kv_pass(p, stream) != cudaSuccess) return FP8Q_ECUDA;
-        }
-        if (crossing != nullptr && !merge) {
-            KvPass q = *crossing;
-            q.early_loads = chained;
-            if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
-        }
-    }
-    const int64_t batches = static_cast<int64_t>(c->batches.size());
-    c->batches.clear();
-    c->used_tokens = 0;
+    // chained: the previous launch on the stream is this call's own amax pass;
+    // the staged rows and the crossing batch were all written before it.
+    const cudaError_t e = fp8q::enqueue_freeze_replay(
+        p, c->stage_k, c->stage_v, c->stage_slots, c->staged_counts.data(),
+        static_cast<int64_t>(c->staged_counts.size()), crossing, chained, stream, &rewritten);
+    if (e != cudaSuccess) return FP8Q_ECUDA;
     c->replayed_tokens = rewritten;
-    c->replayed_batches = batches;
+    c->replayed_batches = static_cast<int64_t>(c->staged_counts.size());
+    c->staged_counts.clear();
+    c->used_tokens = 0;
     c->phase = kFrozen;
     if (replayed) *replayed = rewritten;
     return FP8Q_OK;
@@ -553,7 +472,7 @@ FP8Q_API fp8q_status fp8_kv_calib_restore(fp8_kv_calib *c, float k_scale, float 
                                            as_stream(stream));
     if (e != cudaSuccess) return FP8Q_ECUDA;
     c->phase = kFrozen;
-    c->batches.clear();
+    c->staged_counts.clear();
     c->used_tokens = 0;
     return FP8Q_OK;
 }

@@ -125,6 +125,26 @@ constexpr int64_t kMaxMergedCrossing = 8192;
 constexpr int64_t kMaxLastWriterTokens = 2048;
 bool can_merge_crossing(const KvPass &p);
 
+// The device work of a freeze: every staged batch (packed rows in arrival
+// order, counts[i] rows for batch i, at stage_k / stage_v / stage_slots) is
+// rewritten at the scales frozen from the device maxima, the first launch also
+// publishing them; then `crossing` (the batch that reached the window, a
+// write pass that reads the published scales), if given.  When the window is
+// small enough, every staged row and the crossing batch share one launch that
+// writes each slot only from its last writer; otherwise the batches replay one
+// launch each in arrival order, the last one sharing its launch with the
+// crossing batch when that fits.  Either way each slot ends with its last
+// writer in arrival order.  `base` carries the pools, their geometry,
+// freeze_amax, headroom and scale_out.  `chained`: the launch before this
+// sequence on the stream is a kernel of this library enqueued by the same
+// call (see KvPass::early_loads).  Used by the calibrator and by the
+// allocation-free window call, so both issue the same launches.
+cudaError_t enqueue_freeze_replay(const KvPass &base, const uint16_t *stage_k,
+                                  const uint16_t *stage_v, const int64_t *stage_slots,
+                                  const int64_t *counts, int64_t num_batches,
+                                  const KvPass *crossing, bool chained, cudaStream_t stream,
+                                  int64_t *rewritten);
+
 // Group quantization with phantom rows m..m_pad-1 zeroed and the scales
 // written K-major, scales_km[g * m_pad + r].
 cudaError_t launch_group_quant_kmajor(const uint16_t *x, int64_t x_row_stride, uint8_t *q,

@@ -1136,6 +1136,90 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
     return cudaErrorInvalidValue;
 }
 
+cudaError_t enqueue_freeze_replay(const KvPass &base, const uint16_t *stage_k,
+                                  const uint16_t *stage_v, const int64_t *stage_slots,
+                                  const int64_t *counts, int64_t num_batches,
+                                  const KvPass *crossing, bool chained, cudaStream_t stream,
+                                  int64_t *rewritten) {
+    KvPass p = base;
+    p.do_write = true;
+    p.key_stride = p.elems;   // staging rows are packed
+    p.value_stride = p.elems;
+    p.early_loads = chained;
+
+    int64_t used = 0, last = -1, with_rows = 0;
+    for (int64_t i = 0; i < num_batches; ++i) {
+        used += counts[i];
+        if (counts[i] > 0) {
+            last = i;
+            ++with_rows;
+        }
+    }
+    KvPass probe = p;
+    if (crossing != nullptr) probe.x_tokens = crossing->num_tokens;
+    const bool merge = crossing != nullptr && crossing->num_tokens > 0 &&
+                       crossing->elems == p.elems && can_merge_crossing(probe);
+    auto with_crossing = [&](KvPass q) {
+        q.xk = crossing->k;
+        q.xv = crossing->v;
+        q.x_key_stride = crossing->key_stride;
+        q.x_value_stride = crossing->value_stride;
+        q.x_slots = crossing->slot_mapping;
+        q.x_tokens = crossing->num_tokens;
+        return q;
+    };
+    auto crossing_alone = [&]() {
+        KvPass x = *crossing;
+        x.early_loads = chained;
+        return launch_kv_pass(x, stream);
+    };
+    cudaError_t e = cudaSuccess;
+    *rewritten = 0;
+
+    const int64_t whole_rows = used + (merge ? crossing->num_tokens : 0);
+    if (with_rows >= 2 && whole_rows <= kMaxLastWriterTokens && p.num_slots <= 0x7FFFFFFF) {
+        // the whole window in one launch, each slot from its last writer
+        KvPass q = merge ? with_crossing(p) : p;
+        q.k = stage_k;
+        q.v = stage_v;
+        q.slot_mapping = stage_slots;
+        q.num_tokens = used;
+        q.last_writer = true;
+        if ((e = launch_kv_pass(q, stream)) != cudaSuccess) return e;
+        *rewritten = used;
+        if (crossing != nullptr && !merge) return crossing_alone();
+        return cudaSuccess;
+    }
+    if (merge && last < 0) {
+        // nothing staged with rows: the crossing batch alone, publishing the scales
+        KvPass q = with_crossing(p);
+        q.num_tokens = 0;
+        return launch_kv_pass(q, stream);
+    }
+    bool published = false;
+    int64_t off = 0;
+    for (int64_t i = 0; i < num_batches; ++i) {
+        const int64_t n = counts[i];
+        if (n > 0 || !published) {
+            p.k = stage_k + off * p.elems;
+            p.v = stage_v + off * p.elems;
+            p.slot_mapping = stage_slots + off;
+            p.num_tokens = n;
+            const KvPass q = (merge && i == last) ? with_crossing(p) : p;
+            if ((e = launch_kv_pass(q, stream)) != cudaSuccess) return e;
+            *rewritten += n;
+            published = true;
+        }
+        off += n;
+    }
+    if (!published) {
+        p.num_tokens = 0;
+        if ((e = launch_kv_pass(p, stream)) != cudaSuccess) return e;
+    }
+    if (crossing != nullptr && !merge) return crossing_alone();
+    return cudaSuccess;
+}
+
 cudaError_t launch_kv_write_layers(const KvLayers &p, cudaStream_t stream) {
     if (p.num_tokens == 0 || p.num_layers == 0) return cudaSuccess;
     auto kernel = p.elems == 512 ? kv_write_layers_kernel<64> : kv_write_layers_kernel<0>;

@@ -165,62 +165,23 @@ extern "C" FP8Q_API fp8q_status fp8_kv_calib_window_noalloc(
             if (fp8q::launch_kv_pass(p, stream) != cudaSuccess) return FP8Q_ECUDA;
             stage_row += n;
         } else if (b == freeze_at) {
-            // the batch that reaches the window: its absmax first ...
+            // the batch that reaches the window: its absmax first, then the
+            // freeze with the crossing batch written last, exactly as the
+            // calibrator's fused observe issues them
             fp8q::KvPass a = p;
             a.do_write = false;
             a.do_amax = true;
             a.amax_bits = reinterpret_cast<uint32_t *>(state);
             if (fp8q::launch_kv_pass(a, stream) != cudaSuccess) return FP8Q_ECUDA;
-            // ... then the freeze and the replay of the staged batches, in order ...
             fp8q::KvPass r = w;
-            r.key_stride = elems;
-            r.value_stride = elems;
             r.freeze_amax = reinterpret_cast<uint32_t *>(state);
             r.headroom = h;
             r.scale_out = state + 2;
-            int32_t with_rows = 0;
-            for (int32_t s2 = 0; s2 < b; ++s2) with_rows += batch_tokens[s2] > 0;
-            if (with_rows >= 2 && n > 0 && staged + n <= fp8q::kMaxLastWriterTokens &&
-                w.num_slots <= 0x7FFFFFFF) {
-                // ... all of it in one launch, the crossing batch's rows last and
-                // every slot written by its last writer
-                fp8q::KvPass q = r;
-                q.k = stage_k;
-                q.v = stage_v;
-                q.slot_mapping = stage_slots;
-                q.num_tokens = staged;
-                q.xk = p.k;
-                q.xv = p.v;
-                q.x_key_stride = key_stride;
-                q.x_value_stride = value_stride;
-                q.x_slots = p.slot_mapping;
-                q.x_tokens = n;
-                q.last_writer = true;
-                if (fp8q::launch_kv_pass(q, stream) != cudaSuccess) return FP8Q_ECUDA;
-                row += n;
-                continue;
-            }
-            bool published = false;
-            int64_t off = 0;
-            for (int32_t s = 0; s < b; ++s) {
-                const int64_t m = batch_tokens[s];
-                if (m > 0 || !published) {
-                    r.k = stage_k + off * elems;
-                    r.v = stage_v + off * elems;
-                    r.slot_mapping = stage_slots + off;
-                    r.num_tokens = m;
-                    if (fp8q::launch_kv_pass(r, stream) != cudaSuccess) return FP8Q_ECUDA;
-                    published = true;
-                }
-                off += m;
-            }
-            if (!published) {
-                r.num_tokens = 0;
-                if (fp8q::launch_kv_pass(r, stream) != cudaSuccess) return FP8Q_ECUDA;
-            }
-            // ... then the crossing batch at the frozen scales.
             p.scale_dev = state + 2;
-            if (fp8q::launch_kv_pass(p, stream) != cudaSuccess) return FP8Q_ECUDA;
+            int64_t rewritten = 0;
+            if (fp8q::enqueue_freeze_replay(r, stage_k, stage_v, stage_slots, batch_tokens, b, &p,
+                                            true, stream, &rewritten) != cudaSuccess)
+                return FP8Q_ECUDA;
         } else {
             p.scale_dev = state + 2;
             if (fp8q::launch_kv_pass(p, stream) != cudaSuccess) return FP8Q_ECUDA;

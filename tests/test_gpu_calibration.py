@@ -56,12 +56,19 @@ def _oracle_layer(spec, window, headroom, stage_capacity=None):
     return c, kp, vp
 
 
-def _run_both(spec, batches, window, headroom, fused, stage_capacity=None, check_every=True):
+def _run_both(spec, batches, window, headroom, fused, stage_capacity=None, check_every=True,
+              launches=None):
+    """Drive the GPU layer and the oracle with the same batches; the pools must
+    agree after every batch (or after the last).  ``launches``, if a list,
+    receives the number of kernels the library launched for each batch."""
     g = GpuLayer(spec, window, headroom, fused, stage_capacity)
     c, kp, vp = _oracle_layer(spec, window, headroom, stage_capacity)
     steps = []
     for i, b in enumerate(batches):
+        before = fp8q.launch_count()
         gs = g.step(b)
+        if launches is not None:
+            launches.append(fp8q.launch_count() - before)
         run = cal.run_calibrated_writes(
             c, [cal.KvBatch(b.k, b.v, b.slot_mapping, b.key_stride, b.value_stride)],
             spec.heads, spec.dim, kp, vp, spec.block_size, spec.cache_stride, spec.num_blocks)
@@ -114,31 +121,103 @@ def test_declined_batches(fused):
 
 
 @pytest.mark.parametrize("fused", [False, True])
-def test_crossing_batch_reuses_a_block_of_the_last_staged_batch(fused):
+def test_whole_window_replay_with_the_crossing_batch_on_a_block_of_the_last_staged_batch(fused):
     # batch 9 reaches the window and receives batch 8's second block: the
-    # replay of batch 8 and the crossing write touch the same 16 slots (one
-    # launch in the fused path), and the crossing tokens must end on top
+    # replay of batch 8 and the crossing write touch the same 16 slots.  237
+    # staged rows and 32 crossing rows fit one launch, which writes every slot
+    # from its last writer (the crossing rows come last).
     spec, batches, _ = workloads.calib_window(recycle={6: (2, 1), 9: (8, 1)})
     shared = set(batches[7].slot_mapping) & set(batches[8].slot_mapping)
     assert len(shared) == 16
-    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused)
+    launches = []
+    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused, launches=launches)
     assert steps[8] == fp8q.STEP_FREEZE
+    # fused: absmax + the whole-window launch; unfused: absmax, whole-window
+    # replay, then the crossing batch's own write
+    assert launches[8] == (2 if fused else 3)
     _assert_frozen_state(g, c)
 
 
 @pytest.mark.parametrize("fused", [False, True])
-def test_crossing_set_of_a_pool_above_the_bitmap_limit(fused):
+def test_whole_window_replay_in_a_pool_above_the_bitmap_limit(fused):
     # the same window and block reuse in a pool of 19200 blocks (307200 slots,
-    # above the 2^18 slots a crossing bitmap covers): the merged launch keeps
-    # the crossing slots in its hash set instead
+    # above the 2^18 slots of a crossing bitmap); the whole-window launch keys
+    # its last-writer table by slot whatever the pool size
     spec, batches, _ = workloads.calib_window(recycle={6: (2, 1), 9: (8, 1)})
     big = workloads.PoolSpec(19200, spec.block_size, spec.heads, spec.dim)
     assert big.num_slots > 2 ** 18
     shift = 19000 * spec.block_size
     moved = [workloads.KvBatchInput(b.k, b.v, b.slot_mapping + shift, b.key_stride,
                                     b.value_stride) for b in batches]
-    g, c, steps = _run_both(big, moved, workloads.CALIB_WINDOW, 1.0, fused, check_every=False)
+    launches = []
+    g, c, steps = _run_both(big, moved, workloads.CALIB_WINDOW, 1.0, fused, check_every=False,
+                            launches=launches)
     assert steps[8] == fp8q.STEP_FREEZE
+    assert launches[8] == (2 if fused else 3)
+    _assert_frozen_state(g, c)
+
+
+def _large_window(num_blocks):
+    """Two staged batches of 1000 and 1500 tokens (2500 staged rows, more than
+    one whole-window launch takes) and a 2000-token batch that reaches the
+    4096-token window; its first block is the sixth block of batch 2, so the
+    last staged batch and the crossing batch share 16 slots."""
+    spec, batches, blocks = workloads.calib_window(batch_sizes=(1000, 1500, 2000),
+                                                   recycle={3: (2, 5)}, num_blocks=num_blocks)
+    shared = set(batches[1].slot_mapping) & set(batches[2].slot_mapping)
+    assert len(shared) == 16
+    return spec, batches
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_merged_launch_skips_staged_rows_the_crossing_batch_rewrites(fused):
+    """Per-batch replay with the crossing batch merged into the last staged
+    batch's launch, crossing slots kept as a bitmap over the 8192-slot pool:
+    the 16 staged rows whose slots the crossing batch writes must not land on
+    top of it ("last writer wins", staging.rs module doc)."""
+    spec, batches = _large_window(512)
+    assert spec.num_slots <= 2 ** 18
+    launches = []
+    g, c, steps = _run_both(spec, batches, 4096, 1.0, fused, launches=launches)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
+    # fused: absmax, batch 1's replay, batch 2's replay merged with the
+    # crossing batch; unfused: absmax, two replays, the crossing write
+    assert launches[2] == (3 if fused else 4)
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_merged_launch_hash_set_in_a_pool_above_the_bitmap_limit(fused):
+    """The same window in a pool of 19200 blocks (307200 slots): the merged
+    launch keeps the crossing slots in its shared-memory hash set."""
+    spec, batches = _large_window(19200)
+    assert spec.num_slots > 2 ** 18
+    launches = []
+    g, c, steps = _run_both(spec, batches, 4096, 1.0, fused, check_every=False,
+                            launches=launches)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
+    assert launches[2] == (3 if fused else 4)
+    _assert_frozen_state(g, c)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_window_of_4096_tokens_in_32_token_batches(fused):
+    """A decode-like window: 127 staged batches of 32 tokens (4064 rows), the
+    128th batch reaches 4096, two more follow at the frozen scale.  Batch 10's
+    second block is freed and re-allocated to batch 64, and the crossing batch
+    receives batch 127's first block.  The replay is one launch per staged
+    batch, in arrival order, the last one merged with the crossing batch."""
+    spec, batches, _ = workloads.calib_window(batch_sizes=(32,) * 130,
+                                              recycle={64: (10, 1), 128: (127, 0)},
+                                              num_blocks=512)
+    assert len(set(batches[9].slot_mapping) & set(batches[63].slot_mapping)) == 16
+    assert len(set(batches[126].slot_mapping) & set(batches[127].slot_mapping)) == 16
+    launches = []
+    g, c, steps = _run_both(spec, batches, 4096, 1.0, fused, launches=launches)
+    assert steps == [fp8q.STEP_STAGE] * 127 + [fp8q.STEP_FREEZE] + [fp8q.STEP_FROZEN] * 2
+    assert launches[127] == (1 + 127 if fused else 1 + 127 + 1)
+    assert g.cal.stats()["replayed_batches"] == 127
+    assert g.cal.stats()["replayed_tokens"] == 4064
     _assert_frozen_state(g, c)
 
 
