@@ -181,6 +181,99 @@ class ClockSampler:
                 "samples": len(rows), "window": "warm-up and timed steps"}
 
 
+NVML_POLLER = r"""
+import signal, sys, time
+import pynvml as nv
+signal.signal(signal.SIGTERM, lambda *a: sys.exit(0))
+nv.nvmlInit()
+h = nv.nvmlDeviceGetHandleByUUID(sys.argv[1])
+end = time.monotonic() + float(sys.argv[3])
+with open(sys.argv[2], "w") as out:
+    print("max", nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM), flush=True)
+    while time.monotonic() < end:
+        t = time.monotonic()
+        out.write(f"{t} {nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)} "
+                  f"{nv.nvmlDeviceGetCurrentClocksEventReasons(h)} {nv.nvmlDeviceGetPowerUsage(h)}\n")
+        time.sleep(0.0002)
+"""
+
+
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons of this rank's GPU, polled about
+    every 0.2 ms by a separate process (so the polling never waits for this
+    process's interpreter) and time-stamped on the host's monotonic clock; the
+    samples inside [mark_start, mark_end] are the timed region's.  A timed
+    region of a few milliseconds still gets samples, which a 100 ms
+    nvidia-smi period misses."""
+
+    REASONS = (("gpu_idle", 0x1), ("applications_clocks_setting", 0x2),
+               ("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sync_boost", 0x10),
+               ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("hw_power_brake_slowdown", 0x80), ("display_clock_setting", 0x100))
+
+    def __init__(self, device, max_seconds: float = 600.0) -> None:
+        self.t0 = self.t1 = None
+        self.proc = None
+        self.error = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            fd, self.path = tempfile.mkstemp(prefix="fp8q_nvml_", suffix=".txt")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                [sys.executable, "-c", NVML_POLLER, uuid, self.path, str(max_seconds)],
+                stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+            first = self.proc.stdout.readline().split()   # waits until NVML is up
+            if len(first) != 2 or first[0] != "max":
+                raise RuntimeError("NVML poller did not start: " + self.proc.stderr.read()[-300:])
+            self.max_mhz = int(first[1])
+        except Exception as exc:
+            self.error = f"{type(exc).__name__}: {exc}"
+            if self.proc is not None:
+                self.proc.kill()
+            self.proc = None
+
+    def mark_start(self) -> None:
+        self.t0 = time.monotonic()
+
+    def mark_end(self) -> None:
+        self.t1 = time.monotonic()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"error": self.error or "NVML unavailable"}
+        self.proc.terminate()
+        try:
+            self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.proc.communicate()
+        with open(self.path) as fh:
+            lines = fh.read().splitlines()
+        os.unlink(self.path)
+        rows = []
+        for line in lines:
+            parts = line.split()
+            if len(parts) != 4:
+                continue
+            try:
+                t, sm, r, pw = float(parts[0]), int(parts[1]), int(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            if self.t0 is not None and self.t1 is not None and self.t0 <= t <= self.t1:
+                rows.append((sm, r, pw / 1e3))
+        if not rows:
+            return {"error": "no samples in the timed region", "samples": 0}
+        mask = 0
+        for _, r, _ in rows:
+            mask |= r
+        return {"sm_mhz": statistics.median(c for c, _, _ in rows), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(c for c, _, _ in rows),
+                "power_w_max": round(max(p for _, _, p in rows), 1),
+                "reasons": [name for name, bit in self.REASONS if mask & bit],
+                "samples": len(rows), "timed_region_s": round(self.t1 - self.t0, 4),
+                "window": "timed steps only (NVML in a separate process, ~0.2 ms period)"}
+
+
 # ---------------------------------------------------------------------------
 # the native step
 
@@ -381,15 +474,23 @@ def run_native(args, dist: Dist) -> dict | None:
     assert launches == len(labels), (launches, len(labels))
 
     clocks = ClockSampler(smi_gpu_id(dist.local_rank)) if dist.rank == 0 else None
+    nvml_clocks = NvmlClockSampler(device) if dist.rank == 0 else None
     time_graph(w, stream, graph, args.warmup, reset_state=True)
     torch.cuda.synchronize()
 
     dist.barrier()
     torch.cuda.synchronize()
+    if nvml_clocks is not None:
+        nvml_clocks.mark_start()
     step_ms = time_graph(w, stream, graph, args.steps, reset_state=True)
     torch.cuda.synchronize()
+    if nvml_clocks is not None:
+        nvml_clocks.mark_end()
     dist.barrier()
-    clock_info = clocks.stop() if clocks is not None else None
+    smi_info = clocks.stop() if clocks is not None else None
+    clock_info = nvml_clocks.stop() if nvml_clocks is not None else None
+    if clock_info is not None:
+        clock_info["nvidia_smi_warmup_and_timed"] = smi_info
     gpu_launches = launches * args.steps
 
     total_s = sum(step_ms) / 1e3
@@ -426,6 +527,10 @@ def run_native(args, dist: Dist) -> dict | None:
     drained_ms = drained_step_ms(w, stream, graph, reps=max(20, min(args.steps, 200)))
     seq = kernel_sequences(w, stream, reps=max(5, min(args.steps, 50)))
     targets = measure_targets(w, stream, args)
+    sweep = calib = None
+    if dist.rank == 0 and not args.no_configs:
+        sweep = decode_sweep(device, stream)
+        calib = calib_window(device, stream, warmup=args.warmup, windows=max(10, min(args.steps, 50)))
     e2e = None if args.no_e2e else measure_e2e(w, stream, args)
     del graph
     for c in graph_calibs:
@@ -488,6 +593,10 @@ def run_native(args, dist: Dist) -> dict | None:
         }
         if e2e is not None:
             result["e2e"] = e2e
+        if sweep is not None:
+            result["sweep"] = sweep
+        if calib is not None:
+            result["calib_window"] = calib
         if not args.no_cpu_baseline and dist.world == 1:
             result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
     dist.close()
@@ -495,17 +604,48 @@ def run_native(args, dist: Dist) -> dict | None:
 
 
 def measure_targets(w: Workload, stream, args) -> dict:
-    """The two stand-alone kernel figures the path is judged by: group quant of
+    """The stand-alone kernel figures the path is judged by: group quant of
     the 4593 x 5120 activation (one launch alone, and four back to back on
-    distinct activations), and the steady-state (post-freeze) KV write of 4593
-    tokens per layer, 16 layers back to back (one launch each)."""
+    distinct activations), the K-major variant, and the steady-state
+    (post-freeze) KV write of 4593 tokens per layer, 16 layers back to back
+    (one launch each) and as one multi-layer launch.
+
+    Each figure is given twice: the graph of the launches between CUDA
+    events, and "drained": the same graph followed, inside the timed region,
+    by a read of a clean 2x-L2 buffer that evicts every dirty line the
+    launches left in L2, minus that read on a clean L2.  The drained figure
+    counts the write-back of the codes to HBM, which the plain figure can
+    leave to whatever runs next."""
     fp8q = w.fp8q
     peaks = measured_peaks()
     out = {}
     scale = torch.tensor([0.05, 0.05], dtype=torch.float32, device=w.device)
     reps = max(3, min(args.steps, 50))
+    drain = torch.ones_like(w.flush_read)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def timed(fn, n_launch):
+    def drained_us(g) -> float:
+        with_wb, without = [], []
+        with torch.cuda.stream(stream):
+            for i in range(max(10, reps)):
+                w.flush(i)
+                ev0.record()
+                g.replay()
+                torch.amax(drain)
+                ev1.record()
+                ev1.synchronize()
+                with_wb.append(ev0.elapsed_time(ev1))
+                w.flush(i)
+                ev0.record()
+                torch.amax(drain)
+                ev1.record()
+                ev1.synchronize()
+                without.append(ev0.elapsed_time(ev1))
+        return 1e3 * (statistics.mean(with_wb) - statistics.mean(without))
+
+    drained = {}
+
+    def timed(fn, n_launch, name):
         with torch.cuda.stream(stream):
             fn(lambda i: None)
         torch.cuda.synchronize()
@@ -513,20 +653,34 @@ def measure_targets(w: Workload, stream, args) -> dict:
         with torch.cuda.graph(g, stream=stream):
             fn(lambda i: None)
         ts = time_graph(w, stream, g, reps, reset_state=False)
+        drained[name] = drained_us(g) / n_launch
         del g
         return statistics.mean(ts) * 1e3 / n_launch
+
+    def with_drained(entry, name, nbytes):
+        us = drained[name]
+        gbs = nbytes / (us * 1e-6) / 1e9
+        entry["drained_us"] = round(us, 3)
+        entry["drained_frac_of_hbm"] = round(gbs / peaks["hbm_gbs"], 4)
+        return entry
 
     def gq(mark):
         fp8q.fp8_group_quant(w.x, w.q, w.s)
         mark(0)
 
-    us = timed(gq, 1)
+    us = timed(gq, 1, "gq")
     gbs = GROUP_QUANT_BYTES / (us * 1e-6) / 1e9
-    out["group_quant_4593x5120"] = {"us": round(us, 3), "gbs": round(gbs, 1),
-                                    "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                                    "tokens_per_s": round(M / (us * 1e-6), 1),
-                                    "vs_pages_h100_636_gbs": round(gbs / 636.0, 2),
-                                    "launch": "single launch in its own graph"}
+    out["group_quant_4593x5120"] = with_drained(
+        {"us": round(us, 3), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+         "tokens_per_s": round(M / (us * 1e-6), 1),
+         "vs_pages_h100_636_gbs": round(gbs / 636.0, 2),
+         "launch": "single launch in its own graph"}, "gq", GROUP_QUANT_BYTES)
+    ncu_us = committed_ncu("group_quant", "gpu_time_us")
+    if ncu_us is not None:
+        kgbs = GROUP_QUANT_BYTES / (ncu_us * 1e-6) / 1e9
+        out["group_quant_4593x5120"]["kernel_only"] = {
+            "us": ncu_us, "frac_of_hbm": round(kgbs / peaks["hbm_gbs"], 4),
+            "source": "ncu gpu__time_duration.sum of this launch (profiles/traffic.json)"}
 
     # the fixed cost of this way of timing one launch: the same quantizer on a
     # single 128-element group (one CTA), in its own graph, timed the same way
@@ -538,7 +692,7 @@ def measure_targets(w: Workload, stream, args) -> dict:
         fp8q.fp8_group_quant(x1, q1, s1)
         mark(0)
 
-    out["launch_floor_1x128"] = {"us": round(timed(gq1, 1), 3),
+    out["launch_floor_1x128"] = {"us": round(timed(gq1, 1, "gq1"), 3),
                                  "launch": "single launch in its own graph, one 128-element group"}
 
     # back to back over four distinct activations (as consecutive layers
@@ -552,11 +706,11 @@ def measure_targets(w: Workload, stream, args) -> dict:
             fp8q.fp8_group_quant(xs[i], qs[i], ss[i])
             mark(i)
 
-    us4 = timed(gq4, 4)
+    us4 = timed(gq4, 4, "gq4")
     gbs4 = GROUP_QUANT_BYTES / (us4 * 1e-6) / 1e9
-    out["group_quant_4593x5120_seq4"] = {"us": round(us4, 3), "gbs": round(gbs4, 1),
-                                         "frac_of_hbm": round(gbs4 / peaks["hbm_gbs"], 4),
-                                         "launch": "mean of 4 back-to-back launches"}
+    out["group_quant_4593x5120_seq4"] = with_drained(
+        {"us": round(us4, 3), "gbs": round(gbs4, 1), "frac_of_hbm": round(gbs4 / peaks["hbm_gbs"], 4),
+         "launch": "mean of 4 back-to-back launches"}, "gq4", GROUP_QUANT_BYTES)
     del xs, qs, ss
 
     # the same activation for a GEMM padded to ceil16(M) rows: K-major scales
@@ -569,13 +723,12 @@ def measure_targets(w: Workload, stream, args) -> dict:
         fp8q.fp8_group_quant_kmajor(w.x, m_pad, qk, sk)
         mark(0)
 
-    usk = timed(gqk, 1)
+    usk = timed(gqk, 1, "gqk")
     bk = M * K * 2 + m_pad * K + m_pad * (K // 128) * 4
     gbsk = bk / (usk * 1e-6) / 1e9
-    out["group_quant_kmajor_4593x5120"] = {"us": round(usk, 3), "gbs": round(gbsk, 1),
-                                           "frac_of_hbm": round(gbsk / peaks["hbm_gbs"], 4),
-                                           "m_pad": m_pad, "bytes": bk,
-                                           "launch": "single launch in its own graph"}
+    out["group_quant_kmajor_4593x5120"] = with_drained(
+        {"us": round(usk, 3), "gbs": round(gbsk, 1), "frac_of_hbm": round(gbsk / peaks["hbm_gbs"], 4),
+         "m_pad": m_pad, "bytes": bk, "launch": "single launch in its own graph"}, "gqk", bk)
     del qk, sk
 
     def kvw(mark):
@@ -584,27 +737,26 @@ def measure_targets(w: Workload, stream, args) -> dict:
                               scale_dev=scale)
             mark(l)
 
-    us = timed(kvw, w.layers)
+    us = timed(kvw, w.layers, "kvw")
     b = PER_TOKEN["kv_write"] * TOKENS
     gbs = b / (us * 1e-6) / 1e9
-    out["kv_write_4593"] = {"us_per_layer": round(us, 3), "gbs": round(gbs, 1),
-                            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                            "tokens_per_s": round(TOKENS / (us * 1e-6), 1),
-                            "bytes_per_layer": b,
-                            "launch": f"one launch per layer, {w.layers} back to back"}
+    out["kv_write_4593"] = with_drained(
+        {"us_per_layer": round(us, 3), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+         "tokens_per_s": round(TOKENS / (us * 1e-6), 1), "bytes_per_layer": b,
+         "launch": f"one launch per layer, {w.layers} back to back"}, "kvw", b)
 
     def kvw_layers(mark):
         fp8q.fp8_kv_write_layers(w.k, w.v, w.slots, w.k_pool, w.v_pool,
                                  scale_devs=[scale] * w.layers)
         mark(0)
 
-    us = timed(kvw_layers, 1)
+    us = timed(kvw_layers, 1, "kvl")
     gbs = b * w.layers / (us * 1e-6) / 1e9
-    out["kv_write_4593_all_layers"] = {"us": round(us, 3), "us_per_layer": round(us / w.layers, 3),
-                                       "gbs": round(gbs, 1),
-                                       "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                                       "bytes": b * w.layers,
-                                       "launch": f"fp8_kv_write_layers: {w.layers} layers, one launch"}
+    out["kv_write_4593_all_layers"] = with_drained(
+        {"us": round(us, 3), "us_per_layer": round(us / w.layers, 3), "gbs": round(gbs, 1),
+         "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes": b * w.layers,
+         "launch": f"fp8_kv_write_layers: {w.layers} layers, one launch"}, "kvl", b * w.layers)
+    del drain
     return out
 
 
@@ -736,9 +888,10 @@ KERNEL_OF_LABEL = {
 }
 
 
-def committed_traffic(label: str):
-    """DRAM bytes per launch of `label` from the committed ncu summary, or None
-    when the kernels changed since it was taken."""
+def committed_ncu(label: str, key: str):
+    """A figure of `label`'s launch from the committed ncu summary
+    (profiles/traffic.json), or None when the kernels changed since it was
+    taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as fh:
@@ -748,7 +901,12 @@ def committed_traffic(label: str):
     if t.get("source_hash") != source_hash():
         return None
     entry = t.get("kernels", {}).get(label)
-    return None if entry is None else entry.get("dram_bytes_per_launch")
+    return None if entry is None else entry.get(key)
+
+
+def committed_traffic(label: str):
+    """DRAM bytes per launch of `label` (ncu), or None (see committed_ncu)."""
+    return committed_ncu(label, "dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
@@ -841,7 +999,7 @@ def run_reference(args) -> dict | None:
     }
 
 
-def run_sweep(args) -> list[dict]:
+def decode_sweep(dev, stream, n: int = 1000) -> dict:
     """Decode-width sweep: group quant at M in {1,2,4,8,16} x K in {5120,16384},
     1000 back-to-back launches per shape, timed as plain stream launches
     through the binding and as a CUDA graph of 1000 launches; once with the
@@ -849,11 +1007,7 @@ def run_sweep(args) -> list[dict]:
     zeroed (the layout a padded FP8 GEMM reads).  Launch-bound by design;
     inputs stay in L2, as they do in a decode loop."""
     import paged_kv_cache_group_b200 as fp8q
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
-    stream = torch.cuda.Stream()
-    n = 1000
-    out = []
+    shapes = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for layout in ("row_major", "kmajor"):
         for m in workloads.DECODE_MS:
@@ -896,22 +1050,25 @@ def run_sweep(args) -> list[dict]:
                 # bytes read and written, phantom rows' zero codes and scales included
                 b = m * k * 2 + rows * k + rows * (k // 128) * 4
                 us_p, us_g = statistics.median(plain), statistics.median(graph)
-                out.append({"layout": layout, "m": m, "m_pad": rows, "k": k, "bytes": b,
-                            "plain_us_per_launch": round(us_p, 3),
-                            "graph_us_per_launch": round(us_g, 3),
-                            "graph_gbs": round(b / (us_g * 1e-6) / 1e9, 1),
-                            "graph_tokens_per_s": round(m / (us_g * 1e-6), 1)})
-    return out
+                shapes.append({"layout": layout, "m": m, "m_pad": rows, "k": k, "bytes": b,
+                               "plain_us_per_launch": round(us_p, 3),
+                               "graph_us_per_launch": round(us_g, 3),
+                               "graph_gbs": round(b / (us_g * 1e-6) / 1e9, 1),
+                               "graph_tokens_per_s": round(m / (us_g * 1e-6), 1)})
+    rm = [x["graph_us_per_launch"] for x in shapes if x["layout"] == "row_major"]
+    return {"workload": ("decode-width group quant: M in {1,2,4,8,16} x K in {5120,16384} bf16 "
+                         "N(0,1), groups of 128, 1000 back-to-back launches per shape"),
+            "launches_per_shape": n, "l2": "inputs L2-resident (launch-bound by design)",
+            "row_major_graph_us_per_launch": [min(rm), max(rm)], "shapes": shapes}
 
 
-def run_calib(args) -> dict:
+def calib_window(dev, stream, warmup: int = 5, windows: int = 20) -> dict:
     """The 256-token calibration window of one layer (13 + 32-token batches,
     freeze at batch 9, two batches after it) through fp8_kv_calib_observe_write,
     eager, with L2 flushed before each window; CUDA events around the window."""
     import paged_kv_cache_group_b200 as fp8q
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
     spec, batches, _ = workloads.calib_window()
+
     def rows(bits):
         t = bits.shape[0]
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev).view(t, 4, 128)
@@ -925,20 +1082,22 @@ def run_calib(args) -> dict:
     flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(2 * l2, dtype=torch.uint8, device=dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    stream = torch.cuda.Stream()
     times = []
+    launches = 0
     with torch.cuda.stream(stream):
-        for i in range(args.warmup + args.steps):
+        for i in range(warmup + windows):
             cal = fp8q.KvCalibration(workloads.CALIB_WINDOW, 1.0, 4, 128, dev)
             flush_w.fill_(i & 0xFF)
             torch.amax(flush_r)
             torch.cuda._sleep(1_000_000)       # let the host queue the window ahead
+            before = fp8q.launch_count()
             start.record()
             for k, v, s in zip(ks, vs, ss):
                 cal.observe_write(k, v, s, kp, vp)
             end.record()
+            launches = fp8q.launch_count() - before
             end.synchronize()
-            if i >= args.warmup:
+            if i >= warmup:
                 times.append(start.elapsed_time(end) * 1e3)
             cal.close()
     staged = sum(b.num_tokens for b in batches[:8])
@@ -947,9 +1106,12 @@ def run_calib(args) -> dict:
               (staged + batches[8].num_tokens) * 3080 +
               sum(b.num_tokens for b in batches[9:]) * 3080)
     us = statistics.median(times)
-    return {"workload": "calibration window: 256 tokens, 4 x 128, batches 13 + 10 x 32",
-            "us_per_window": round(us, 2), "tokens": seen, "bytes": bytes_,
-            "gbs": round(bytes_ / (us * 1e-6) / 1e9, 1), "windows": len(times)}
+    return {"workload": ("calibration window: 256 tokens, 4 x 128, batches 13 + 10 x 32, freeze at "
+                         "batch 9 (269 tokens), headroom 1.0"),
+            "us_per_window": round(us, 2), "tokens": seen, "bytes": bytes_, "launches": launches,
+            "gbs": round(bytes_ / (us * 1e-6) / 1e9, 1),
+            "tokens_per_s": round(seen / (us * 1e-6), 1), "windows": len(times),
+            "l2": "flushed before each window", "timing": "CUDA events around the window's calls"}
 
 
 def run_profile(args) -> None:
@@ -991,6 +1153,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--layers", type=int, default=workloads.LARGE_LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the decode-width sweep and the calibration window")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--profile", action="store_true",
@@ -1012,12 +1176,15 @@ def main(argv=None) -> int:
     if args.profile:
         run_profile(args)
         return 0
-    if args.sweep:
-        for line in run_sweep(args):
-            print(json.dumps(line), flush=True)
-        return 0
-    if args.calib:
-        print(json.dumps(run_calib(args)), flush=True)
+    if args.sweep or args.calib:
+        torch.cuda.set_device(0)
+        dev = torch.device("cuda", 0)
+        stream = torch.cuda.Stream(dev)
+        if args.sweep:
+            for line in decode_sweep(dev, stream)["shapes"]:
+                print(json.dumps(line), flush=True)
+        if args.calib:
+            print(json.dumps(calib_window(dev, stream, args.warmup, args.steps)), flush=True)
         return 0
     if args.impl == "reference":
         res = run_reference(args)
