@@ -249,7 +249,10 @@ struct TensorEncoder {
     bool scaled;         // r >= 1: take the product on r' and scale back
     bool ok;             // scale is a positive number
 
-    __device__ __forceinline__ void init(float scale) {
+    // `bounded`: the caller knows |x| / s <= 448 for every x it encodes (the
+    // maxima the scale comes from cover them), so x * r cannot overflow and
+    // the plain form serves.
+    __device__ __forceinline__ void init(float scale, bool bounded = false) {
         s = scale;
         ok = s > 0.0f;   // false for NaN
         fast = (s >= 0x1p-64f) && (s <= 0x1p64f);
@@ -257,22 +260,30 @@ struct TensorEncoder {
         const float r = __frcp_rn(s);
         pd.r2 = pair(r, r);
         pd.ns2 = pair(-s, -s);
-        // r' = r * 2^-k in [0.5, 1), s' = s * 2^k, c = 2^k: exponent-field
-        // arithmetic, exact for the normal r and s of the fast range
-        const int k = r >= 1.0f ? static_cast<int>((__float_as_uint(r) >> 23) & 0xFF) - 126 : 0;
-        scaled = k > 0;
-        const float rs = __uint_as_float(__float_as_uint(r) - (static_cast<uint32_t>(k) << 23));
-        const float ss = __uint_as_float(__float_as_uint(s) + (static_cast<uint32_t>(k) << 23));
-        const float c = __uint_as_float(static_cast<uint32_t>(127 + k) << 23);
-        sd.rs2 = pair(rs, rs);
-        sd.nss2 = pair(-ss, -ss);
-        sd.c2 = pair(c, c);
-        sd.r2 = pd.r2;
+        scaled = !bounded && fast && !pow2 && r >= 1.0f;
+        if (scaled) {
+            // r' = r * 2^-k in [0.5, 1), s' = s * 2^k, c = 2^k: exponent-field
+            // arithmetic, exact for the normal r and s of the fast range
+            const uint32_t k = ((__float_as_uint(r) >> 23) & 0xFF) - 126;
+            const float rs = __uint_as_float(__float_as_uint(r) - (k << 23));
+            const float ss = __uint_as_float(__float_as_uint(s) + (k << 23));
+            const float c = __uint_as_float((127 + k) << 23);
+            sd.rs2 = pair(rs, rs);
+            sd.nss2 = pair(-ss, -ss);
+            sd.c2 = pair(c, c);
+            sd.r2 = pd.r2;
+        }
     }
 
-    // The caller knows |x| / s <= 448 for every x it encodes (the maxima the
-    // scale comes from cover them): x * r cannot overflow, so the plain form.
-    __device__ __forceinline__ void within_range() { scaled = false; }
+    // The calibrator's provisional scale 2.0 (in-window writes): a power of
+    // two, r = 0.5 exactly, no reciprocal to compute.
+    __device__ __forceinline__ void init_provisional() {
+        s = 2.0f;
+        ok = fast = pow2 = true;
+        scaled = false;
+        pd.r2 = pair(0.5f, 0.5f);
+        pd.ns2 = pair(-2.0f, -2.0f);
+    }
 
     // Two chunks of a row.
     __device__ __forceinline__ void encode2(const uint4 &a, const uint4 &b, uint2 &oa,
@@ -588,15 +599,10 @@ __device__ __forceinline__ void resolve_scales(const KvPass &p, TensorEncoder &k
         ks = p.k_scale;
         vs = p.v_scale;
     }
-    kenc.init(ks);
-    venc.init(vs);
-    if (p.freeze_amax != nullptr) {
-        // Every row a freeze pass writes (staged or crossing) went into the
-        // maxima the scale comes from, so |x| / s <= 448 / headroom <= 448 and
-        // x * r cannot overflow.
-        kenc.within_range();
-        venc.within_range();
-    }
+    // Every row a freeze pass writes (staged or crossing) went into the maxima
+    // the scale comes from, so |x| / s <= 448 / headroom <= 448.
+    kenc.init(ks, p.freeze_amax != nullptr);
+    venc.init(vs, p.freeze_amax != nullptr);
     if (!(kenc.ok && venc.ok) && blockIdx.x == 0 && threadIdx.x == 0)
         atomicOr(&g_error_word, kErrScale);
 }
@@ -846,7 +852,14 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) kv_pass_kernel(cons
         allow_next_grid();
     }
     TensorEncoder kenc, venc;
-    if (kWrite) resolve_scales(p, kenc, venc);
+    if (kWrite && kAmax) {
+        // a write in the same pass as the absmax is an in-window write, always
+        // at the provisional scale (launch_kv_pass checks it)
+        kenc.init_provisional();
+        venc.init_provisional();
+    } else if (kWrite) {
+        resolve_scales(p, kenc, venc);
+    }
 
     const bool small_slots = p.num_slots <= 0x7FFFFFFF;
     uint32_t kacc = 0, vacc = 0;
@@ -897,6 +910,87 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) kv_pass_kernel(cons
             if (vm) atomicMax(p.amax_bits + 1, vm << 16);
         }
     }
+}
+
+// Byte offset of this lane's first 8 codes in the pool entry of `slot`, or -1
+// for a slot that is skipped (padding, or out of range: reported).
+__device__ __forceinline__ int64_t entry512(const KvPass &p, int64_t slot, int lane) {
+    if (slot < 0) return -1;
+    if (slot >= p.num_slots) {
+        if (lane == 0) atomicOr(&g_error_word, kErrSlot);
+        return -1;
+    }
+    int64_t blk, off;
+    if (p.block_shift >= 0) {
+        blk = slot >> p.block_shift;
+        off = slot & ((int64_t{1} << p.block_shift) - 1);
+    } else if (p.num_slots <= 0x7FFFFFFF) {
+        const uint32_t s32 = static_cast<uint32_t>(slot);
+        const uint32_t b32 = s32 / static_cast<uint32_t>(p.block_size);
+        blk = b32;
+        off = s32 - b32 * static_cast<uint32_t>(p.block_size);
+    } else {
+        blk = slot / p.block_size;
+        off = slot - blk * p.block_size;
+    }
+    return blk * p.cache_stride + off * 512 + lane * 8;
+}
+
+// This lane's 16 values of one row (chunks a and b) into the pool at `dst`.
+__device__ __forceinline__ void write_half512(uint8_t *pool, int64_t dst, const uint4 &a,
+                                              const uint4 &b, const TensorEncoder &enc) {
+    uint2 oa, ob;
+    enc.encode2(a, b, oa, ob);
+    *reinterpret_cast<uint2 *>(pool + dst) = oa;
+    *reinterpret_cast<uint2 *>(pool + dst + 256) = ob;
+}
+
+// The plain quantize-and-scatter of 512-element rows (4 KV heads x 128, the
+// pages' shape): nothing but the write, one token per warp and a grid that
+// covers every token (575 CTAs of 256 threads for a 4593-token layer, in one
+// wave).  The K half is encoded and stored before the V encoder is set up,
+// so only one encoder's constants are held at a time.  Same lane mapping
+// and encode as the general pass, without its switches; kEarly is
+// KvPass::early_loads.  Measured in chains of 16 4593-token layers on one
+// box: 3.85 us per layer (general pass, two tokens per warp) -> 3.59 us; two
+// tokens per warp on 256- or 512-thread CTAs came out at 3.72-3.81 us.
+template <bool kEarly>
+__global__ void __launch_bounds__(kKvThreads, 4) kv_write512_kernel(const KvPass p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
+    const bool have = t < p.num_tokens;
+    if (!kEarly) {
+        // this token's K row (lane 0) and V row (lane 1) into L2 while the
+        // previous kernel finishes
+        if (lane < 2 && have) prefetch_row<false>(p, t, lane);
+        wait_for_previous_grid();
+        allow_next_grid();
+    }
+    Row r;
+    if (have) load_row<false, true, 64>(p, t, lane, 64, r);
+    if (kEarly) {
+        wait_for_previous_grid();
+        allow_next_grid();
+    }
+    float ks = p.k_scale, vs = p.v_scale;
+    if (p.scale_dev != nullptr) {
+        const float2 sd = *reinterpret_cast<const float2 *>(p.scale_dev);
+        ks = sd.x;
+        vs = sd.y;
+    }
+    if (!(ks > 0.0f && vs > 0.0f) && blockIdx.x == 0 && threadIdx.x == 0)
+        atomicOr(&g_error_word, kErrScale);
+    if (!have) return;
+    const int64_t d = entry512(p, r.slot, lane);
+    if (d < 0) return;
+    {
+        TensorEncoder enc;
+        enc.init(ks);
+        if (enc.ok) write_half512(p.k_pool, d, r.ka, r.kb, enc);
+    }
+    TensorEncoder enc;
+    enc.init(vs);
+    if (enc.ok) write_half512(p.v_pool, d, r.va, r.vb, enc);
 }
 
 // Many layers' writes in one grid: blockIdx.y is the layer, blockIdx.x walks
@@ -1128,6 +1222,16 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
         return launch_kv_variant<false, false, true, true>(p, stream);
     }
     if (p.num_tokens == 0 && !publish) return cudaSuccess;
+    if (p.do_amax && p.do_write &&
+        (p.k_scale != 2.0f || p.v_scale != 2.0f || p.scale_dev != nullptr ||
+         p.freeze_amax != nullptr))
+        return cudaErrorInvalidValue;   // in-window writes take the provisional scale
+    if (p.do_write && !p.do_amax && !p.do_stage && p.elems == 512 && p.freeze_amax == nullptr) {
+        auto kernel = p.early_loads ? kv_write512_kernel<true> : kv_write512_kernel<false>;
+        const int64_t grid = (p.num_tokens + kKvWarps - 1) / kKvWarps;   // one token per warp
+        if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        return launch(kernel, static_cast<int>(grid), kKvThreads, 0, stream, p);
+    }
     if (p.do_amax && p.do_stage && p.do_write) return launch_kv_variant<true, true, true, false>(p, stream);
     if (p.do_amax && p.do_stage) return launch_kv_variant<true, true, false, false>(p, stream);
     if (p.do_amax && p.do_write) return launch_kv_variant<true, false, true, false>(p, stream);
