@@ -993,6 +993,83 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_write512_kernel(const KvPass
     if (enc.ok) write_half512(p.v_pool, d, r.va, r.vb, enc);
 }
 
+// The merged freeze launch for 512-element rows with the crossing set as a
+// bitmap (pools of at most 2^18 slots): the last staged batch replayed and
+// the crossing batch written, at the scales frozen from the device maxima,
+// one token per warp.  A staged row whose slot the crossing batch also
+// writes is skipped (the crossing row is the later writer).  Same result as
+// the general pass's merged launch, without its switches; the K half of a row
+// is written before the V encoder is set up.  kEarly is KvPass::early_loads:
+// rows are loaded and the bitmap is built before the dependency wait.
+constexpr int kFreezeThreads = 512;
+
+template <bool kEarly>
+__global__ void __launch_bounds__(kFreezeThreads, 2) kv_freeze512_kernel(const KvPass p) {
+    constexpr int kWarps = kFreezeThreads / 32;
+    extern __shared__ uint32_t s_bits[];   // one bit per pool slot: the crossing slots
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * kFreezeThreads + threadIdx.x) >> 5;
+    const int64_t total = p.num_tokens + p.x_tokens;
+    const bool have = t < total;
+    // with one token per warp, a CTA holds staged rows iff its first row is one
+    const bool need_table = static_cast<int64_t>(blockIdx.x) * kWarps < p.num_tokens;
+    if (!kEarly) {
+        if (lane < 2 && have) prefetch_row<true>(p, t, lane);
+        if (need_table && threadIdx.x == 32) {
+            const int64_t bytes = p.x_tokens * 8;
+            if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0)
+                prefetch_l2_bulk(p.x_slots, static_cast<uint32_t>(bytes));
+        }
+        wait_for_previous_grid();
+        allow_next_grid();
+    }
+    Row r;
+    if (have) load_row<true, true, 64>(p, t, lane, 64, r);
+    if (need_table) {
+        const int n4 = static_cast<int>((p.num_slots + 127) >> 7);
+        uint4 *bits4 = reinterpret_cast<uint4 *>(s_bits);
+        for (int i = threadIdx.x; i < n4; i += kFreezeThreads) bits4[i] = make_uint4(0, 0, 0, 0);
+        __syncthreads();
+        for (int64_t i = threadIdx.x; i < p.x_tokens; i += kFreezeThreads) {
+            const int64_t sl = __ldg(p.x_slots + i);
+            if (sl >= 0 && sl < p.num_slots)
+                atomicOr(&s_bits[static_cast<uint32_t>(sl) >> 5],
+                         1u << (static_cast<uint32_t>(sl) & 31u));
+        }
+        __syncthreads();
+    }
+    if (kEarly) {
+        wait_for_previous_grid();
+        allow_next_grid();
+    }
+    const uint2 a = *reinterpret_cast<const uint2 *>(p.freeze_amax);
+    const float ks = freeze_scale(a.x, p.headroom);
+    const float vs = freeze_scale(a.y, p.headroom);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (p.scale_out != nullptr) {
+            p.scale_out[0] = ks;
+            p.scale_out[1] = vs;
+        }
+        if (!(ks > 0.0f && vs > 0.0f)) atomicOr(&g_error_word, kErrScale);
+    }
+    if (!have) return;
+    const int64_t slot = r.slot;
+    if (t < p.num_tokens && slot >= 0 && slot < p.num_slots &&
+        ((s_bits[static_cast<uint32_t>(slot) >> 5] >> (static_cast<uint32_t>(slot) & 31u)) & 1u))
+        return;   // the crossing batch writes this slot later
+    const int64_t d = entry512(p, slot, lane);
+    if (d < 0) return;
+    // every row written here went into the maxima the scales come from
+    {
+        TensorEncoder enc;
+        enc.init(ks, true);
+        if (enc.ok) write_half512(p.k_pool, d, r.ka, r.kb, enc);
+    }
+    TensorEncoder enc;
+    enc.init(vs, true);
+    if (enc.ok) write_half512(p.v_pool, d, r.va, r.vb, enc);
+}
+
 // Many layers' writes in one grid: blockIdx.y is the layer, blockIdx.x walks
 // that layer's tokens.  Per CTA, thread 0 resolves the layer's scales; the
 // rows go through the same code as a one-layer write.
@@ -1219,6 +1296,13 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
     const bool cross = p.do_write && p.x_tokens > 0;
     if (cross) {
         if (!can_merge_crossing(p) || p.do_amax || p.do_stage) return cudaErrorInvalidValue;
+        if (p.elems == 512 && p.freeze_amax != nullptr && p.num_slots <= kBitmapMaxSlots) {
+            auto kernel = p.early_loads ? kv_freeze512_kernel<true> : kv_freeze512_kernel<false>;
+            const int64_t grid = (p.num_tokens + p.x_tokens + kFreezeThreads / 32 - 1) /
+                                 (kFreezeThreads / 32);
+            const size_t smem = static_cast<size_t>((p.num_slots + 127) >> 7) * 16;
+            return launch(kernel, static_cast<int>(grid), kFreezeThreads, smem, stream, p);
+        }
         return launch_kv_variant<false, false, true, true>(p, stream);
     }
     if (p.num_tokens == 0 && !publish) return cudaSuccess;
