@@ -993,6 +993,70 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_write512_kernel(const KvPass
     if (enc.ok) write_half512(p.v_pool, d, r.va, r.vb, enc);
 }
 
+// The in-window pass for 512-element rows: the batch's |K| and |V| maxima
+// max-accumulated into the device state, its rows copied (packed) to staging
+// with their slots, and its rows written at the provisional scale 2.0, all
+// from one read of K and V, one token per warp.  Same result as the general
+// pass with all three jobs, without its switches.  kEarly is
+// KvPass::early_loads.
+template <bool kEarly>
+__global__ void __launch_bounds__(kKvThreads, 4) kv_stage512_kernel(const KvPass p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
+    const bool have = t < p.num_tokens;
+    if (!kEarly) {
+        if (lane < 2 && have) prefetch_row<false>(p, t, lane);
+        wait_for_previous_grid();
+        allow_next_grid();
+    }
+    Row r;
+    uint32_t kacc = 0, vacc = 0;
+    if (have) {
+        load_row<false, true, 64>(p, t, lane, 64, r);
+        kacc = absmax_uint4(absmax_uint4(kacc, r.ka), r.kb);
+        vacc = absmax_uint4(absmax_uint4(vacc, r.va), r.vb);
+    }
+    if (kEarly) {
+        wait_for_previous_grid();
+        allow_next_grid();
+    }
+    if (have) {
+        const int64_t row = (p.stage_offset + t) * 512 + lane * 8;
+        *reinterpret_cast<uint4 *>(p.stage_k + row) = r.ka;
+        *reinterpret_cast<uint4 *>(p.stage_k + row + 256) = r.kb;
+        *reinterpret_cast<uint4 *>(p.stage_v + row) = r.va;
+        *reinterpret_cast<uint4 *>(p.stage_v + row + 256) = r.vb;
+        if (lane == 0) p.stage_slots[p.stage_offset + t] = r.slot;
+        const int64_t d = entry512(p, r.slot, lane);
+        if (d >= 0) {
+            TensorEncoder enc;
+            enc.init_provisional();
+            write_half512(p.k_pool, d, r.ka, r.kb, enc);
+            write_half512(p.v_pool, d, r.va, r.vb, enc);
+        }
+    }
+    __shared__ uint32_t red[2][kKvWarps];
+    const uint32_t km = __reduce_max_sync(0xFFFFFFFFu, absmax_bits16(kacc));
+    const uint32_t vm = __reduce_max_sync(0xFFFFFFFFu, absmax_bits16(vacc));
+    const int w = threadIdx.x >> 5;
+    if (lane == 0) {
+        red[0][w] = km;
+        red[1][w] = vm;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t k = red[0][0], v = red[1][0];
+#pragma unroll
+        for (int i = 1; i < kKvWarps; ++i) {
+            k = max(k, red[0][i]);
+            v = max(v, red[1][i]);
+        }
+        // fp32 bit patterns of non-negative values order like unsigned integers
+        if (k) atomicMax(p.amax_bits + 0, k << 16);
+        if (v) atomicMax(p.amax_bits + 1, v << 16);
+    }
+}
+
 // The merged freeze launch for 512-element rows with the crossing set as a
 // bitmap (pools of at most 2^18 slots): the last staged batch replayed and
 // the crossing batch written, at the scales frozen from the device maxima,
@@ -1310,6 +1374,12 @@ cudaError_t launch_kv_pass(const KvPass &p, cudaStream_t stream) {
         (p.k_scale != 2.0f || p.v_scale != 2.0f || p.scale_dev != nullptr ||
          p.freeze_amax != nullptr))
         return cudaErrorInvalidValue;   // in-window writes take the provisional scale
+    if (p.do_amax && p.do_stage && p.do_write && p.elems == 512) {
+        auto kernel = p.early_loads ? kv_stage512_kernel<true> : kv_stage512_kernel<false>;
+        const int64_t grid = (p.num_tokens + kKvWarps - 1) / kKvWarps;   // one token per warp
+        if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        return launch(kernel, static_cast<int>(grid), kKvThreads, 0, stream, p);
+    }
     if (p.do_write && !p.do_amax && !p.do_stage && p.elems == 512 && p.freeze_amax == nullptr) {
         auto kernel = p.early_loads ? kv_write512_kernel<true> : kv_write512_kernel<false>;
         const int64_t grid = (p.num_tokens + kKvWarps - 1) / kKvWarps;   // one token per warp
