@@ -880,11 +880,12 @@ def source_hash() -> str:
 # ncu kernel of each bench label (the launch list names kernels, not labels)
 KERNEL_OF_LABEL = {
     "group_quant": "group_quant_kernel<1>",
-    "observe_stage_write": "kv_pass_kernel<1, 1, 1, 0, 64, 256>",
+    "observe_stage_write": "kv_stage512_kernel<0>",
     "amax": "kv_pass_kernel<1, 0, 0, 0, 64, 256>",
-    "replay_crossing": "kv_pass_kernel<0, 0, 1, 1, 64, 512>",
-    "kv_write": "kv_pass_kernel<0, 0, 1, 0, 64, 256>",
+    "replay_crossing": "kv_freeze512_kernel<1>",
+    "kv_write": "kv_write512_kernel<0>",
     "kv_write_layers": "kv_write_layers_kernel<64>",
+    "group_quant_kmajor": "group_quant_kmajor_kernel",
 }
 
 

@@ -461,17 +461,20 @@ group_quant_kmajor_kernel(const uint16_t *__restrict__ x, int64_t x_row_stride,
 // ---------------------------------------------------------------------------
 // 2./3. KV pass: absmax, staging copy and quantize-and-scatter
 //
-// One warp per token (grid-stride; the plain write takes two tokens per warp
-// on half the grid).  Lane l owns 16-byte chunks l and l+32 of the K row and
+// One warp per token.  Lane l owns 16-byte chunks l and l+32 of the K row and
 // of the V row, so every load and store instruction of the warp is one
 // contiguous run (512 B of bf16 in, 256 B of codes out).  The slot decides
 // where the codes land: one token's entry is E contiguous bytes of the pool,
 // written as 32 8-byte stores per instruction.
 //
-// Each warp issues its first token's loads before anything else, then
-// resolves the scales itself (a dependent 8-byte load; for a freeze the frozen
-// scale from the device maxima) while those loads are in flight.  CTAs are 256
-// threads, 512 for the merged freeze launch (see kv_pass_kernel).
+// Each warp issues its token's loads before anything else, then resolves the
+// scales itself (a dependent 8-byte load; for a freeze the frozen scale from
+// the device maxima) while those loads are in flight.  CTAs are 256 threads,
+// 512 for the merged freeze launch.  Rows of 4 x 128 elements (the pages'
+// shape) take kernels of their own for the three passes of the calibrating
+// write path (kv_stage512_kernel, kv_freeze512_kernel, kv_write512_kernel);
+// kv_pass_kernel serves every other shape and job (grid-stride when the
+// batch is larger than the resident grid).
 
 constexpr int kKvThreads = 256;
 constexpr int kKvWarps = kKvThreads / 32;
@@ -770,20 +773,11 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) kv_pass_kernel(cons
     // A whole-window replay checks every row against its last-writer table.
     const bool need_table =
         kCross && (p.last_writer || static_cast<int64_t>(blockIdx.x) * kWarps < p.num_tokens);
-    // The plain write takes two tokens per warp (half the grid, so the next
-    // launch's CTAs fit beside this one's and can prefetch early); both rows
-    // are prefetched before the wait and loaded together.
-    constexpr bool kTwo = kWrite && !kAmax && !kStage && !kCross;
     const bool early = p.early_loads;
     if (!early) {
         // the first token's K row, V row and slot into L2 while the previous
         // kernel finishes (and, for a merged crossing batch, its slot list)
-        if (kTwo) {
-            const int64_t tt = warp + (lane >> 1) * nwarps;
-            if (lane < 4 && tt < total) prefetch_row<kCross>(p, tt, lane & 1);
-        } else if (warp < total && lane < 2) {
-            prefetch_row<kCross>(p, warp, lane);
-        }
+        if (warp < total && lane < 2) prefetch_row<kCross>(p, warp, lane);
         if (need_table && threadIdx.x == 32) {
             const int64_t bytes = p.x_tokens * 8;
             if ((reinterpret_cast<uintptr_t>(p.x_slots) & 15) == 0 && bytes % 16 == 0 &&
@@ -866,17 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) kv_pass_kernel(cons
 
     // the first token (the only one unless the grid is smaller than the
     // batch), then the rest of the grid-stride loop
-    if (kTwo && t + nwarps < total) {
-        Row r2;
-        load_row<kCross, kSlot, kChunks>(p, t + nwarps, lane, nchunks, r2);
-        process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
-                                                            s_table, log2, small_slots, kacc,
-                                                            vacc);
-        t += nwarps;
-        process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r2, t, lane, nchunks, kenc, venc,
-                                                            s_table, log2, small_slots, kacc,
-                                                            vacc);
-    } else if (t < total) {
+    if (t < total) {
         process_row<kAmax, kStage, kWrite, kCross, kChunks>(p, r, t, lane, nchunks, kenc, venc,
                                                             s_table, log2, small_slots, kacc,
                                                             vacc);
@@ -952,8 +936,9 @@ __device__ __forceinline__ void write_half512(uint8_t *pool, int64_t dst, const 
 // so only one encoder's constants are held at a time.  Same lane mapping
 // and encode as the general pass, without its switches; kEarly is
 // KvPass::early_loads.  Measured in chains of 16 4593-token layers on one
-// box: 3.85 us per layer (general pass, two tokens per warp) -> 3.59 us; two
-// tokens per warp on 256- or 512-thread CTAs came out at 3.72-3.81 us.
+// box: 3.85 us per layer (general pass, then with two tokens per warp) ->
+// 3.59 us; two tokens per warp on 256- or 512-thread CTAs came out at
+// 3.72-3.81 us.
 template <bool kEarly>
 __global__ void __launch_bounds__(kKvThreads, 4) kv_write512_kernel(const KvPass p) {
     const int lane = threadIdx.x & 31;
@@ -1299,8 +1284,7 @@ cudaError_t launch_kv_variant(const KvPass &p, cudaStream_t stream) {
     auto kernel = p.elems == 512 ? kv_pass_kernel<A, S, W, X, 64, kThreads>
                                  : kv_pass_kernel<A, S, W, X, 0, kThreads>;
     const int64_t tokens = p.num_tokens + (X ? p.x_tokens : 0);
-    const int64_t per_cta = (W && !A && !S && !X) ? 2 * kWarps : kWarps;   // see kTwo
-    const int64_t wanted = (tokens + per_cta - 1) / per_cta;
+    const int64_t wanted = (tokens + kWarps - 1) / kWarps;
     const size_t smem =
         !X ? 0
            : p.last_writer ? (size_t{8} << last_writer_log2(tokens))

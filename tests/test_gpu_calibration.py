@@ -297,6 +297,26 @@ def test_large_prefill_single_chunk_freezes_at_once(fused):
     _assert_frozen_state(g, c)
 
 
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("heads,dim", [(2, 64), (8, 128)])
+def test_calibration_window_with_other_row_widths(fused, heads, dim):
+    """Rows of 128 and 1024 elements take the general passes (the workload's
+    512-element rows have kernels of their own): the in-window pass, the
+    whole-window replay, and the merged launch of one staged batch with the
+    crossing batch."""
+    spec, batches, _ = workloads.calib_window(heads=heads, dim=dim)
+    g, c, steps = _run_both(spec, batches, workloads.CALIB_WINDOW, 1.0, fused)
+    assert steps == [fp8q.STEP_STAGE] * 8 + [fp8q.STEP_FREEZE] + [fp8q.STEP_FROZEN] * 2
+    _assert_frozen_state(g, c)
+    spec, batches, _ = workloads.calib_window(batch_sizes=(13, 32, 32), heads=heads, dim=dim)
+    launches = []
+    g, c, steps = _run_both(spec, batches, 20, 1.0, fused, launches=launches)
+    assert steps == [fp8q.STEP_STAGE, fp8q.STEP_FREEZE, fp8q.STEP_FROZEN]
+    # fused: absmax + the merged launch; unfused: absmax, replay, crossing write
+    assert launches[1] == (2 if fused else 3)
+    _assert_frozen_state(g, c)
+
+
 def test_zero_token_observe_counts_a_stage_step():
     spec, batches, _ = workloads.calib_window(batch_sizes=(13, 32))
     empty = workloads.KvBatchInput(batches[0].k[:0], batches[0].v[:0],

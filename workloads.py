@@ -186,16 +186,17 @@ CALIB_BATCHES = (13,) + (32,) * 10   # 8 staged, batch 9 crosses, 2 after
 
 
 def calib_window(batch_sizes=CALIB_BATCHES, row_pad: int = 0, recycle=None,
-                 num_blocks: int = 128):
+                 num_blocks: int = 128, heads: int = KV_HEADS, dim: int = HEAD_DIM):
     """Calibration-window workload: returns (spec, batches, blocks per batch).
 
     ``recycle`` maps a batch number to (earlier batch number, block index):
     before that batch, the earlier batch's block is freed and is the first
     block the batch receives.  The default reuses batch 2's second block in
     batch 6.  ``num_blocks`` sizes the pool (128 blocks of 16 slots for the
-    256-token window; larger windows need a larger pool)."""
+    256-token window; larger windows need a larger pool); ``heads`` x ``dim``
+    is the row shape (4 x 128 in the workload)."""
     recycle = {6: (2, 1)} if recycle is None else recycle
-    spec = PoolSpec(num_blocks, 16, KV_HEADS, HEAD_DIM)
+    spec = PoolSpec(num_blocks, 16, heads, dim)
     g = generator(CALIB, 0, 0)
     alloc = BlockAllocator(spec.num_blocks, generator(CALIB, 0, 1))
     batches = []
