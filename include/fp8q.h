@@ -403,8 +403,10 @@ FP8Q_API fp8q_status fp8_kv_freeze_replay(fp8_kv_calib *calib, void *k_pool,
  * fp8_kv_write at the scales the step calls for (and, on FP8Q_STEP_FREEZE,
  * fp8_kv_freeze_replay in between), with identical results.  In the window
  * the absmax, the staging copy and the provisional-scale write share one
- * read of K and V; on the freeze the absmax, the replay and the crossing
- * write are three stream-ordered launches; after it, one write.
+ * read of K and V; on the freeze the absmax comes first, then the replay,
+ * whose last launch also writes the crossing batch when it fits (a crossing
+ * batch above 8192 tokens gets a launch of its own after it); after the
+ * freeze, one write.
  * Returns as fp8_kv_calib_observe and fp8_kv_freeze_replay.
  */
 FP8Q_API fp8q_status fp8_kv_calib_observe_write(

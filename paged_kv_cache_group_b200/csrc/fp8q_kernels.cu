@@ -32,9 +32,7 @@
 
 #include <atomic>
 #include <cstdint>
-#include <map>
 #include <mutex>
-#include <tuple>
 #include <utility>
 
 #include "fp8q_internal.h"
@@ -1215,30 +1213,42 @@ cudaError_t device_sms(int *sms) {
 }
 
 // Resident CTAs per SM of a kernel at a dynamic shared-memory size, cached
-// per (device, kernel, size).
+// per (device, kernel, size) in a fixed table: no launch path allocates, host
+// or device (a full table only means the query is repeated).
+struct OccEntry {
+    int dev;
+    const void *kernel;
+    size_t smem;
+    int ctas;
+};
+constexpr int kOccEntries = 512;
 std::mutex g_occ_mutex;
-std::map<std::tuple<int, const void *, size_t>, int> g_occ;
+OccEntry g_occ[kOccEntries];
+int g_occ_used = 0;
 
 template <typename Kernel>
 cudaError_t resident_ctas(Kernel kernel, int threads, size_t smem, int *out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const auto key = std::make_tuple(dev, reinterpret_cast<const void *>(kernel), smem);
+    const void *key = reinterpret_cast<const void *>(kernel);
     std::lock_guard<std::mutex> lock(g_occ_mutex);
-    auto it = g_occ.find(key);
-    if (it == g_occ.end()) {
-        if (smem > 48 * 1024) {
-            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem));
-            if (e != cudaSuccess) return e;
+    for (int i = 0; i < g_occ_used; ++i) {
+        if (g_occ[i].dev == dev && g_occ[i].kernel == key && g_occ[i].smem == smem) {
+            *out = g_occ[i].ctas;
+            return cudaSuccess;
         }
-        int n = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
-        if (e != cudaSuccess) return e;
-        it = g_occ.emplace(key, n > 0 ? n : 1).first;
     }
-    *out = it->second;
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+    if (e != cudaSuccess) return e;
+    *out = n > 0 ? n : 1;
+    if (g_occ_used < kOccEntries) g_occ[g_occ_used++] = OccEntry{dev, key, smem, *out};
     return cudaSuccess;
 }
 
