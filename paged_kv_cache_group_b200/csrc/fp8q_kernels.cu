@@ -1047,7 +1047,12 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_stage512_kernel(const KvPass
 // writes is skipped (the crossing row is the later writer).  Same result as
 // the general pass's merged launch, without its switches; the K half of a row
 // is written before the V encoder is set up.  kEarly is KvPass::early_loads:
-// rows are loaded and the bitmap is built before the dependency wait.
+// the row and this thread's first crossing slots are loaded before the
+// dependency wait.  After the wait the device maxima are loaded and the
+// bitmap is built while that load is in flight, so the table adds no memory
+// latency of its own (measured per 4593-row launch: 3.96 -> 3.63-3.74 us;
+// building the table before the wait put the slot loads and the maxima load
+// one after the other).
 constexpr int kFreezeThreads = 512;
 
 template <bool kEarly>
@@ -1072,24 +1077,35 @@ __global__ void __launch_bounds__(kFreezeThreads, 2) kv_freeze512_kernel(const K
     }
     Row r;
     if (have) load_row<true, true, 64>(p, t, lane, 64, r);
+    // this thread's first two crossing slots, loaded with its row
+    int64_t s0 = -1, s1 = -1;
     if (need_table) {
-        const int n4 = static_cast<int>((p.num_slots + 127) >> 7);
-        uint4 *bits4 = reinterpret_cast<uint4 *>(s_bits);
-        for (int i = threadIdx.x; i < n4; i += kFreezeThreads) bits4[i] = make_uint4(0, 0, 0, 0);
-        __syncthreads();
-        for (int64_t i = threadIdx.x; i < p.x_tokens; i += kFreezeThreads) {
-            const int64_t sl = __ldg(p.x_slots + i);
-            if (sl >= 0 && sl < p.num_slots)
-                atomicOr(&s_bits[static_cast<uint32_t>(sl) >> 5],
-                         1u << (static_cast<uint32_t>(sl) & 31u));
-        }
-        __syncthreads();
+        const int64_t i0 = threadIdx.x, i1 = threadIdx.x + kFreezeThreads;
+        if (i0 < p.x_tokens) s0 = __ldg(p.x_slots + i0);
+        if (i1 < p.x_tokens) s1 = __ldg(p.x_slots + i1);
     }
     if (kEarly) {
         wait_for_previous_grid();
         allow_next_grid();
     }
+    // the device maxima, in flight while the bitmap is built
     const uint2 a = *reinterpret_cast<const uint2 *>(p.freeze_amax);
+    if (need_table) {
+        const int n4 = static_cast<int>((p.num_slots + 127) >> 7);
+        uint4 *bits4 = reinterpret_cast<uint4 *>(s_bits);
+        for (int i = threadIdx.x; i < n4; i += kFreezeThreads) bits4[i] = make_uint4(0, 0, 0, 0);
+        __syncthreads();
+        auto insert = [&](int64_t sl) {
+            if (sl >= 0 && sl < p.num_slots)
+                atomicOr(&s_bits[static_cast<uint32_t>(sl) >> 5],
+                         1u << (static_cast<uint32_t>(sl) & 31u));
+        };
+        insert(s0);
+        insert(s1);
+        for (int64_t i = threadIdx.x + 2 * kFreezeThreads; i < p.x_tokens; i += kFreezeThreads)
+            insert(__ldg(p.x_slots + i));
+        __syncthreads();
+    }
     const float ks = freeze_scale(a.x, p.headroom);
     const float vs = freeze_scale(a.y, p.headroom);
     if (blockIdx.x == 0 && threadIdx.x == 0) {

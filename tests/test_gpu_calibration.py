@@ -157,12 +157,12 @@ def test_whole_window_replay_in_a_pool_above_the_bitmap_limit(fused):
     _assert_frozen_state(g, c)
 
 
-def _large_window(num_blocks):
+def _large_window(num_blocks, crossing=2000):
     """Two staged batches of 1000 and 1500 tokens (2500 staged rows, more than
-    one whole-window launch takes) and a 2000-token batch that reaches the
-    4096-token window; its first block is the sixth block of batch 2, so the
-    last staged batch and the crossing batch share 16 slots."""
-    spec, batches, blocks = workloads.calib_window(batch_sizes=(1000, 1500, 2000),
+    one whole-window launch takes) and a batch of ``crossing`` tokens that
+    reaches the 2501-token window; its first block is the sixth block of batch
+    2, so the last staged batch and the crossing batch share 16 slots."""
+    spec, batches, blocks = workloads.calib_window(batch_sizes=(1000, 1500, crossing),
                                                    recycle={3: (2, 5)}, num_blocks=num_blocks)
     shared = set(batches[1].slot_mapping) & set(batches[2].slot_mapping)
     assert len(shared) == 16
@@ -170,15 +170,18 @@ def _large_window(num_blocks):
 
 
 @pytest.mark.parametrize("fused", [False, True])
-def test_merged_launch_skips_staged_rows_the_crossing_batch_rewrites(fused):
+@pytest.mark.parametrize("crossing", [500, 2000])
+def test_merged_launch_skips_staged_rows_the_crossing_batch_rewrites(fused, crossing):
     """Per-batch replay with the crossing batch merged into the last staged
-    batch's launch, crossing slots kept as a bitmap over the 8192-slot pool:
-    the 16 staged rows whose slots the crossing batch writes must not land on
-    top of it ("last writer wins", staging.rs module doc)."""
-    spec, batches = _large_window(512)
+    batch's launch: the 16 staged rows whose slots the crossing batch writes
+    must not land on top of it ("last writer wins", staging.rs module doc).
+    500 crossing rows: each staged row's warp compares its slot with the
+    crossing slots; 2000: the crossing slots as a bitmap over the 8192-slot
+    pool."""
+    spec, batches = _large_window(512, crossing)
     assert spec.num_slots <= 2 ** 18
     launches = []
-    g, c, steps = _run_both(spec, batches, 4096, 1.0, fused, launches=launches)
+    g, c, steps = _run_both(spec, batches, 2501, 1.0, fused, launches=launches)
     assert steps == [fp8q.STEP_STAGE, fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
     # fused: absmax, batch 1's replay, batch 2's replay merged with the
     # crossing batch; unfused: absmax, two replays, the crossing write
@@ -193,7 +196,7 @@ def test_merged_launch_hash_set_in_a_pool_above_the_bitmap_limit(fused):
     spec, batches = _large_window(19200)
     assert spec.num_slots > 2 ** 18
     launches = []
-    g, c, steps = _run_both(spec, batches, 4096, 1.0, fused, check_every=False,
+    g, c, steps = _run_both(spec, batches, 2501, 1.0, fused, check_every=False,
                             launches=launches)
     assert steps == [fp8q.STEP_STAGE, fp8q.STEP_STAGE, fp8q.STEP_FREEZE]
     assert launches[2] == (3 if fused else 4)
