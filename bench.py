@@ -401,12 +401,13 @@ def drained_step_ms(w: Workload, stream, graph, reps: int) -> float:
             end.synchronize()
             without.append(start.elapsed_time(end))
     del drain, sink
-    return statistics.mean(with_wb) - statistics.mean(without)
+    return statistics.median(with_wb) - statistics.median(without)
 
 
 def kernel_sequences(w: Workload, stream, reps: int) -> dict:
-    """Average launch duration of each kernel of the step, from a graph of its
-    launches exactly as the step issues them (one per layer, back to back),
+    """Launch duration of each kernel of the step (median over the repetitions
+    of a graph of its launches, divided by the launches), the graph issuing
+    them exactly as the step does (one per layer, back to back),
     the state before them prepared eagerly.  The merged freeze launch is only
     reachable together with the crossing chunk's absmax, so its time is the
     difference between that pair's graph and the absmax-only graph.
@@ -444,7 +445,7 @@ def kernel_sequences(w: Workload, stream, reps: int) -> dict:
         del g
         for c in calibs:
             c.close()
-        return 1e3 * statistics.mean(ts)
+        return 1e3 * statistics.median(ts)
 
     gq = timed([], lambda c: fp8q.fp8_group_quant(w.x, w.q, w.s), 1)
     stage = timed([], stage_all, L)
@@ -610,10 +611,10 @@ def measure_targets(w: Workload, stream, args) -> dict:
     (post-freeze) KV write of 4593 tokens per layer, 16 layers back to back
     (one launch each) and as one multi-layer launch.
 
-    Each figure is given twice: the graph of the launches between CUDA
-    events, and "drained": the same graph followed, inside the timed region,
-    by a read of a clean 2x-L2 buffer that evicts every dirty line the
-    launches left in L2, minus that read on a clean L2.  The drained figure
+    Each figure is given twice (medians over the repetitions): the graph of
+    the launches between CUDA events, and "drained": the same graph followed,
+    inside the timed region, by a read of a clean 2x-L2 buffer that evicts
+    every dirty line the launches left in L2, minus that read on a clean L2.  The drained figure
     counts the write-back of the codes to HBM, which the plain figure can
     leave to whatever runs next."""
     fp8q = w.fp8q
@@ -641,7 +642,7 @@ def measure_targets(w: Workload, stream, args) -> dict:
                 ev1.record()
                 ev1.synchronize()
                 without.append(ev0.elapsed_time(ev1))
-        return 1e3 * (statistics.mean(with_wb) - statistics.mean(without))
+        return 1e3 * (statistics.median(with_wb) - statistics.median(without))
 
     drained = {}
 
@@ -655,7 +656,7 @@ def measure_targets(w: Workload, stream, args) -> dict:
         ts = time_graph(w, stream, g, reps, reset_state=False)
         drained[name] = drained_us(g) / n_launch
         del g
-        return statistics.mean(ts) * 1e3 / n_launch
+        return statistics.median(ts) * 1e3 / n_launch
 
     def with_drained(entry, name, nbytes):
         us = drained[name]
