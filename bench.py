@@ -192,8 +192,12 @@ with open(sys.argv[2], "w") as out:
     print("max", nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM), flush=True)
     while time.monotonic() < end:
         t = time.monotonic()
-        out.write(f"{t} {nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)} "
-                  f"{nv.nvmlDeviceGetCurrentClocksEventReasons(h)} {nv.nvmlDeviceGetPowerUsage(h)}\n")
+        try:
+            out.write(f"{t} {nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)} "
+                      f"{nv.nvmlDeviceGetCurrentClocksEventReasons(h)} "
+                      f"{nv.nvmlDeviceGetPowerUsage(h)}\n")
+        except nv.NVMLError as exc:
+            print("nvml", exc, file=sys.stderr, flush=True)
         time.sleep(0.0002)
 """
 
@@ -204,7 +208,9 @@ class NvmlClockSampler:
     process's interpreter) and time-stamped on the host's monotonic clock; the
     samples inside [mark_start, mark_end] are the timed region's.  A timed
     region of a few milliseconds still gets samples, which a 100 ms
-    nvidia-smi period misses."""
+    nvidia-smi period misses.  sample_now() adds one query from this process;
+    the timed loop calls it after enqueuing each step, while the GPU runs it,
+    so the region has samples even when the poller is starved of CPU time."""
 
     REASONS = (("gpu_idle", 0x1), ("applications_clocks_setting", 0x2),
                ("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sync_boost", 0x10),
@@ -231,6 +237,34 @@ class NvmlClockSampler:
             if self.proc is not None:
                 self.proc.kill()
             self.proc = None
+        # the same query from this process, once per timed step while the GPU
+        # works on it, so the region has samples even when the poller process
+        # is not scheduled in time on a busy host
+        self.local = []
+        self.nv = self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(
+                "GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+            if self.proc is None:
+                self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:
+            self.nv = None
+            self.error = (self.error or "") + f" in-process NVML: {type(exc).__name__}: {exc}"
+
+    def sample_now(self) -> None:
+        """One sample from this process (called while a timed step runs)."""
+        if self.nv is None:
+            return
+        nv, h = self.nv, self.handle
+        try:
+            self.local.append((time.monotonic(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                               nv.nvmlDeviceGetCurrentClocksEventReasons(h),
+                               nv.nvmlDeviceGetPowerUsage(h)))
+        except Exception:
+            pass
 
     def mark_start(self) -> None:
         self.t0 = time.monotonic()
@@ -239,18 +273,24 @@ class NvmlClockSampler:
         self.t1 = time.monotonic()
 
     def stop(self) -> dict:
-        if self.proc is None:
+        lines, stderr = [], ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                _, stderr = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                _, stderr = self.proc.communicate()
+            with open(self.path) as fh:
+                lines = fh.read().splitlines()
+            os.unlink(self.path)
+        if self.proc is None and self.nv is None:
             return {"error": self.error or "NVML unavailable"}
-        self.proc.terminate()
-        try:
-            self.proc.communicate(timeout=10)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            self.proc.communicate()
-        with open(self.path) as fh:
-            lines = fh.read().splitlines()
-        os.unlink(self.path)
-        rows = []
+
+        def inside(t):
+            return self.t0 is not None and self.t1 is not None and self.t0 <= t <= self.t1
+
+        rows, poller_rows, poller_total = [], 0, 0
         for line in lines:
             parts = line.split()
             if len(parts) != 4:
@@ -259,10 +299,19 @@ class NvmlClockSampler:
                 t, sm, r, pw = float(parts[0]), int(parts[1]), int(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            if self.t0 is not None and self.t1 is not None and self.t0 <= t <= self.t1:
+            poller_total += 1
+            if inside(t):
                 rows.append((sm, r, pw / 1e3))
+                poller_rows += 1
+        local_rows = 0
+        for t, sm, r, pw in self.local:
+            if inside(t):
+                rows.append((sm, r, pw / 1e3))
+                local_rows += 1
         if not rows:
-            return {"error": "no samples in the timed region", "samples": 0}
+            return {"error": "no samples in the timed region", "samples": 0,
+                    "poller_samples_total": poller_total,
+                    "poller_stderr": (stderr or "")[-300:], "note": self.error}
         mask = 0
         for _, r, _ in rows:
             mask |= r
@@ -270,8 +319,11 @@ class NvmlClockSampler:
                 "sm_mhz_min": min(c for c, _, _ in rows),
                 "power_w_max": round(max(p for _, _, p in rows), 1),
                 "reasons": [name for name, bit in self.REASONS if mask & bit],
-                "samples": len(rows), "timed_region_s": round(self.t1 - self.t0, 4),
-                "window": "timed steps only (NVML in a separate process, ~0.2 ms period)"}
+                "samples": len(rows), "samples_poller": poller_rows,
+                "samples_in_process": local_rows,
+                "timed_region_s": round(self.t1 - self.t0, 4),
+                "window": ("timed steps only: NVML polled every ~0.2 ms by a separate process, "
+                           "plus one in-process query per step while the GPU runs it")}
 
 
 # ---------------------------------------------------------------------------
@@ -359,7 +411,11 @@ def capture(w: Workload, stream):
     return graph, labels, launches, calibs
 
 
-def time_graph(w: Workload, stream, graph, reps: int, reset_state: bool) -> list[float]:
+def time_graph(w: Workload, stream, graph, reps: int, reset_state: bool,
+               during=None) -> list[float]:
+    """Event time of each of reps replays, L2 flushed (and the calibrator
+    state reset when reset_state) before each; during() runs on the host
+    after each replay is enqueued, while the GPU works on it."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     out = []
     with torch.cuda.stream(stream):
@@ -371,6 +427,8 @@ def time_graph(w: Workload, stream, graph, reps: int, reset_state: bool) -> list
             start.record()
             graph.replay()
             end.record()
+            if during is not None:
+                during()
             end.synchronize()
             out.append(start.elapsed_time(end))
     return out
@@ -404,32 +462,62 @@ def drained_step_ms(w: Workload, stream, graph, reps: int) -> float:
     return statistics.median(with_wb) - statistics.median(without)
 
 
+def launch_counts(layers: int) -> list[int]:
+    """Graph sizes (launches per kernel) over which per-launch times are fitted."""
+    return sorted({n for n in (1, 2, 4, 8, layers) if 1 <= n <= layers})
+
+
+def fit_line(points: dict) -> tuple[float, float]:
+    """Least-squares line through {n: t}: (slope, intercept)."""
+    ns = list(points)
+    if len(ns) == 1:
+        return points[ns[0]] / ns[0], 0.0
+    mn = statistics.fmean(ns)
+    mt = statistics.fmean(points.values())
+    slope = (sum((n - mn) * (points[n] - mt) for n in ns) /
+             sum((n - mn) ** 2 for n in ns))
+    return slope, mt - slope * mn
+
+
 def kernel_sequences(w: Workload, stream, reps: int) -> dict:
-    """Launch duration of each kernel of the step (median over the repetitions
-    of a graph of its launches, divided by the launches), the graph issuing
-    them exactly as the step does (one per layer, back to back),
-    the state before them prepared eagerly.  The merged freeze launch is only
-    reachable together with the crossing chunk's absmax, so its time is the
-    difference between that pair's graph and the absmax-only graph.
-    Returns {label: (us per launch, launches per graph)}."""
+    """Launch duration of each kernel of the step.  For each kernel, graphs of
+    n of its launches (n = 1, 2, 4, 8 and all layers, one per layer, back to
+    back as the step issues them, the state before them prepared eagerly;
+    for group quant n = 1, 2, 4, 8 over four activations in turn) are timed
+    between CUDA events (median over the repetitions), and the per-launch
+    duration is the slope of graph time against n.  The intercept
+    is the fixed cost of timing one graph after the L2 flush (about 5 us; a
+    graph of one single-group launch shows the same), which belongs to no
+    launch; graph time / launches at n = all layers is kept beside the slope.
+    The merged freeze launch is only reachable together with the crossing
+    chunk's absmax, so its times are the differences between that pair's
+    graphs and the absmax-only graphs.
+    Returns {label: {"us": slope, "intercept_us", "graph_us_per_launch",
+    "graph_us": {n: us}}}."""
     fp8q = w.fp8q
     L = w.layers
 
-    def stage_all(calibs):
-        for l, c in enumerate(calibs):
-            c.observe_write(w.k[l][:CHUNK1], w.v[l][:CHUNK1], w.slots[l][:CHUNK1],
-                            w.k_pool[l], w.v_pool[l])
+    def stage_n(n):
+        def body(calibs):
+            for l in range(n):
+                calibs[l].observe_write(w.k[l][:CHUNK1], w.v[l][:CHUNK1], w.slots[l][:CHUNK1],
+                                        w.k_pool[l], w.v_pool[l])
+        return body
 
-    def amax_all(calibs):
-        for l, c in enumerate(calibs):
-            c.observe(w.k[l][CHUNK1:], w.v[l][CHUNK1:], w.slots[l][CHUNK1:])
+    def amax_n(n):
+        def body(calibs):
+            for l in range(n):
+                calibs[l].observe(w.k[l][CHUNK1:], w.v[l][CHUNK1:], w.slots[l][CHUNK1:])
+        return body
 
-    def freeze_all(calibs):
-        for l, c in enumerate(calibs):
-            c.observe_write(w.k[l][CHUNK1:], w.v[l][CHUNK1:], w.slots[l][CHUNK1:],
-                            w.k_pool[l], w.v_pool[l])
+    def freeze_n(n):
+        def body(calibs):
+            for l in range(n):
+                calibs[l].observe_write(w.k[l][CHUNK1:], w.v[l][CHUNK1:], w.slots[l][CHUNK1:],
+                                        w.k_pool[l], w.v_pool[l])
+        return body
 
-    def timed(prefix, body, n):
+    def timed(prefix, body, n_launch):
         with torch.cuda.stream(stream):
             w.states.copy_(w.states_init)
             calibs = w.calibrators()
@@ -440,19 +528,42 @@ def kernel_sequences(w: Workload, stream, reps: int) -> dict:
         before = fp8q.launch_count()
         with torch.cuda.graph(g, stream=stream):
             body(calibs)
-        assert fp8q.launch_count() - before == n
+        assert fp8q.launch_count() - before == n_launch
         ts = time_graph(w, stream, g, reps, reset_state=False)
         del g
         for c in calibs:
             c.close()
         return 1e3 * statistics.median(ts)
 
-    gq = timed([], lambda c: fp8q.fp8_group_quant(w.x, w.q, w.s), 1)
-    stage = timed([], stage_all, L)
-    amax = timed([stage_all], amax_all, L)
-    pair = timed([stage_all], freeze_all, 2 * L)
-    return {"group_quant": (gq, 1), "observe_stage_write": (stage / L, L),
-            "amax": (amax / L, L), "replay_crossing": (max(pair - amax, 0.0) / L, L)}
+    ns = launch_counts(L)
+    xs = [w.x] + [w.x.clone() for _ in range(3)]
+    qs = [w.q] + [torch.empty_like(w.q) for _ in range(3)]
+    ss = [w.s] + [torch.empty_like(w.s) for _ in range(3)]
+
+    def gq_n(n):
+        # four distinct activations in turn (4 x 71 MB: a launch's input and
+        # output have left L2 by the time they come round again)
+        def body(calibs):
+            for i in range(n):
+                fp8q.fp8_group_quant(xs[i % 4], qs[i % 4], ss[i % 4])
+        return body
+
+    graphs = {
+        "group_quant": {n: timed([], gq_n(n), n) for n in (1, 2, 4, 8)},
+        "observe_stage_write": {n: timed([], stage_n(n), n) for n in ns},
+        "amax": {n: timed([stage_n(L)], amax_n(n), n) for n in ns},
+    }
+    pair = {n: timed([stage_n(L)], freeze_n(n), 2 * n) for n in ns}
+    graphs["replay_crossing"] = {n: max(pair[n] - graphs["amax"][n], 0.0) for n in ns}
+    del xs, qs, ss
+    out = {}
+    for lab, pts in graphs.items():
+        slope, icept = fit_line(pts)
+        n_max = max(pts)
+        out[lab] = {"us": slope, "intercept_us": icept,
+                    "graph_us_per_launch": pts[n_max] / n_max,
+                    "graph_us": {n: round(t, 3) for n, t in pts.items()}}
+    return out
 
 
 def run_native(args, dist: Dist) -> dict | None:
@@ -483,7 +594,8 @@ def run_native(args, dist: Dist) -> dict | None:
     torch.cuda.synchronize()
     if nvml_clocks is not None:
         nvml_clocks.mark_start()
-    step_ms = time_graph(w, stream, graph, args.steps, reset_state=True)
+    step_ms = time_graph(w, stream, graph, args.steps, reset_state=True,
+                         during=nvml_clocks.sample_now if nvml_clocks is not None else None)
     torch.cuda.synchronize()
     if nvml_clocks is not None:
         nvml_clocks.mark_end()
@@ -540,15 +652,20 @@ def run_native(args, dist: Dist) -> dict | None:
     result = None
     if dist.rank == 0:
         kernels = {}
-        kernel_time = sum(us * labels.count(lab) for lab, (us, _) in seq.items())
-        for lab, (avg_us, _) in seq.items():
+        kernel_time = sum(v["us"] * labels.count(lab) for lab, v in seq.items())
+        for lab, v in seq.items():
             n_per_step = labels.count(lab)
             b = launch_bytes(lab)
-            gbs = b / (avg_us * 1e-6) / 1e9
-            kernels[lab] = {"launches_per_step": n_per_step, "avg_us": round(avg_us, 3),
+            gbs = b / (v["us"] * 1e-6) / 1e9
+            graph_gbs = b / (v["graph_us_per_launch"] * 1e-6) / 1e9
+            kernels[lab] = {"launches_per_step": n_per_step, "avg_us": round(v["us"], 3),
                             "bytes_per_launch": b, "gbs": round(gbs, 1),
                             "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                            "share": round(n_per_step * avg_us / kernel_time, 4)}
+                            "share": round(n_per_step * v["us"] / kernel_time, 4),
+                            "fit_intercept_us": round(v["intercept_us"], 3),
+                            "graph_us_per_launch": round(v["graph_us_per_launch"], 3),
+                            "graph_frac_of_hbm": round(graph_gbs / peaks["hbm_gbs"], 4),
+                            "graph_us_by_launches": v["graph_us"]}
         dominant = max(kernels, key=lambda k: kernels[k]["launches_per_step"] * kernels[k]["avg_us"])
         dk = kernels[dominant]
         ms = 1e3 * max_s / args.steps
@@ -568,7 +685,10 @@ def run_native(args, dist: Dist) -> dict | None:
                 "l2": "flushed before every step (2x L2 write, then 2x L2 read; untimed)",
                 "timing": ("CUDA graph replay of the step's 49 launches (programmatic "
                            "dependent launch), CUDA events around each step; per-kernel "
-                           "times from graphs of each kernel's launches in step order"),
+                           "launch duration = slope of event-timed graph time against "
+                           "launches (graphs of 1, 2, 4, 8 and all layers' launches of that "
+                           "kernel in step order; group quant: 1, 2, 4, 8 launches over four "
+                           "activations); graph time / launches kept beside it"),
                 "bytes_per_step": step_bytes(args.layers),
                 "parallelism": f"replicas x{dist.world} (one step per GPU, no collective)",
             },
@@ -578,7 +698,13 @@ def run_native(args, dist: Dist) -> dict | None:
                          "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4),
                          "traffic": committed_traffic(dominant),
                          "peak_source": peaks["source"],
-                         "algorithmic_bytes_per_launch": dk["bytes_per_launch"]},
+                         "algorithmic_bytes_per_launch": dk["bytes_per_launch"],
+                         "launch_us": dk["avg_us"],
+                         "launch_us_method": ("slope of event-timed graph time against the "
+                                              "number of launches; the intercept, the fixed "
+                                              "cost of timing a graph, is excluded"),
+                         "graph_us_per_launch": dk["graph_us_per_launch"],
+                         "graph_frac": dk["graph_frac_of_hbm"]},
             "kernels": kernels,
             "targets": targets,
             "eager_ms_per_step": round(statistics.median(eager_ms), 4),
@@ -616,7 +742,12 @@ def measure_targets(w: Workload, stream, args) -> dict:
     inside the timed region, by a read of a clean 2x-L2 buffer that evicts
     every dirty line the launches left in L2, minus that read on a clean L2.  The drained figure
     counts the write-back of the codes to HBM, which the plain figure can
-    leave to whatever runs next."""
+    leave to whatever runs next.  The chained figures (group quant, K-major,
+    per-layer KV write) also carry the marginal duration: the slope of graph
+    time against the number of launches, which leaves out the fixed cost of
+    timing a graph between events (about 5 us after the L2 flush; a graph of
+    one single-group launch shows the same) and, in a chain, counts the
+    write-back of the previous launch's codes."""
     fp8q = w.fp8q
     peaks = measured_peaks()
     out = {}
@@ -646,7 +777,7 @@ def measure_targets(w: Workload, stream, args) -> dict:
 
     drained = {}
 
-    def timed(fn, n_launch, name):
+    def timed(fn, n_launch, name, drain_too=True):
         with torch.cuda.stream(stream):
             fn(lambda i: None)
         torch.cuda.synchronize()
@@ -654,9 +785,22 @@ def measure_targets(w: Workload, stream, args) -> dict:
         with torch.cuda.graph(g, stream=stream):
             fn(lambda i: None)
         ts = time_graph(w, stream, g, reps, reset_state=False)
-        drained[name] = drained_us(g) / n_launch
+        if drain_too:
+            drained[name] = drained_us(g) / n_launch
         del g
         return statistics.median(ts) * 1e3 / n_launch
+
+    def marginal(entry, make_fn, ns, nbytes, unit_key):
+        """Slope of graph time against launches (graphs of n launches for n in
+        ns): the per-launch duration without the fixed cost of timing a graph."""
+        pts = {n: timed(make_fn(n), n, f"fit{n}", drain_too=False) * n for n in ns}
+        slope, icept = fit_line(pts)
+        gbs = nbytes / (slope * 1e-6) / 1e9
+        entry[unit_key] = round(slope, 3)
+        entry["marginal_frac_of_hbm"] = round(gbs / peaks["hbm_gbs"], 4)
+        entry["fit_intercept_us"] = round(icept, 3)
+        entry["graph_us_by_launches"] = {n: round(t, 3) for n, t in pts.items()}
+        return entry
 
     def with_drained(entry, name, nbytes):
         us = drained[name]
@@ -712,7 +856,17 @@ def measure_targets(w: Workload, stream, args) -> dict:
     out["group_quant_4593x5120_seq4"] = with_drained(
         {"us": round(us4, 3), "gbs": round(gbs4, 1), "frac_of_hbm": round(gbs4 / peaks["hbm_gbs"], 4),
          "launch": "mean of 4 back-to-back launches"}, "gq4", GROUP_QUANT_BYTES)
-    del xs, qs, ss
+
+    def gq_first(n):
+        def fn(mark):
+            for i in range(n):
+                fp8q.fp8_group_quant(xs[i % 4], qs[i % 4], ss[i % 4])
+                mark(i)
+        return fn
+
+    marginal(out["group_quant_4593x5120_seq4"], gq_first, (1, 2, 4, 8), GROUP_QUANT_BYTES,
+             "marginal_us")
+    del qs, ss
 
     # the same activation for a GEMM padded to ceil16(M) rows: K-major scales
     # and zeroed phantom rows in the same launch
@@ -730,7 +884,18 @@ def measure_targets(w: Workload, stream, args) -> dict:
     out["group_quant_kmajor_4593x5120"] = with_drained(
         {"us": round(usk, 3), "gbs": round(gbsk, 1), "frac_of_hbm": round(gbsk / peaks["hbm_gbs"], 4),
          "m_pad": m_pad, "bytes": bk, "launch": "single launch in its own graph"}, "gqk", bk)
-    del qk, sk
+    qks = [qk] + [torch.empty_like(qk) for _ in range(3)]
+    sks = [sk] + [torch.empty_like(sk) for _ in range(3)]
+
+    def gqk_first(n):
+        def fn(mark):
+            for i in range(n):
+                fp8q.fp8_group_quant_kmajor(xs[i % 4], m_pad, qks[i % 4], sks[i % 4])
+                mark(i)
+        return fn
+
+    marginal(out["group_quant_kmajor_4593x5120"], gqk_first, (1, 2, 4, 8), bk, "marginal_us")
+    del qk, sk, qks, sks, xs
 
     def kvw(mark):
         for l in range(w.layers):
@@ -745,6 +910,16 @@ def measure_targets(w: Workload, stream, args) -> dict:
         {"us_per_layer": round(us, 3), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
          "tokens_per_s": round(TOKENS / (us * 1e-6), 1), "bytes_per_layer": b,
          "launch": f"one launch per layer, {w.layers} back to back"}, "kvw", b)
+
+    def kvw_first(n):
+        def fn(mark):
+            for l in range(n):
+                fp8q.fp8_kv_write(w.k[l], w.v[l], w.slots[l], w.k_pool[l], w.v_pool[l],
+                                  scale_dev=scale)
+                mark(l)
+        return fn
+
+    marginal(out["kv_write_4593"], kvw_first, launch_counts(w.layers), b, "marginal_us_per_layer")
 
     def kvw_layers(mark):
         fp8q.fp8_kv_write_layers(w.k, w.v, w.slots, w.k_pool, w.v_pool,

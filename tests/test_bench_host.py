@@ -1,6 +1,7 @@
 """Host-side logic on CPU: bench.py's multi-rank aggregation (gloo, world
-size 2) and its reference arm's JSON contract, and the all-reduce of the KV
-maxima for heads sharded over ranks (gloo, world size 2)."""
+size 2), its reference arm's JSON contract, the per-launch slope fit and the
+clock-sample window, and the all-reduce of the KV maxima for heads sharded
+over ranks (gloo, world size 2)."""
 import argparse
 import os
 import socket
@@ -82,6 +83,43 @@ def test_algorithmic_bytes():
     assert bench.step_bytes(16) == 71_283_360 + 16 * (4095 * 5136 + 498 * 2048 + 4095 * 3080 +
                                                       498 * 3080)
     assert len(bench.labels_of(16)) == 49
+
+
+def test_launch_counts_cover_one_to_all_layers():
+    assert bench.launch_counts(16) == [1, 2, 4, 8, 16]
+    assert bench.launch_counts(2) == [1, 2]
+    assert bench.launch_counts(1) == [1]
+    assert bench.launch_counts(12) == [1, 2, 4, 8, 12]
+
+
+def test_fit_line_recovers_slope_and_intercept():
+    pts = {n: 5.1 + 3.25 * n for n in (1, 2, 4, 8, 16)}
+    slope, icept = bench.fit_line(pts)
+    assert slope == pytest.approx(3.25) and icept == pytest.approx(5.1)
+    assert bench.fit_line({4: 12.0}) == (3.0, 0.0)
+    # event deltas that snap up to a 2.048 us grid: over 1..16 launches the
+    # slope stays within 2.048 / 15 of the true one
+    tick = 2.048
+    snapped = {n: tick * -(-(5.1 + 3.25 * n) // tick) for n in (1, 2, 4, 8, 16)}
+    slope, _ = bench.fit_line(snapped)
+    assert abs(slope - 3.25) < tick / 15
+
+
+def test_clock_samples_outside_the_timed_region_are_dropped():
+    smp = object.__new__(bench.NvmlClockSampler)
+    smp.proc, smp.nv, smp.error, smp.max_mhz = None, object(), None, 1965
+    smp.t0, smp.t1 = 10.0, 11.0
+    smp.local = [(9.5, 900, 0x1, 90_000),          # before: idle clock, not counted
+                 (10.2, 1965, 0x0, 600_000),
+                 (10.7, 1900, 0x4, 980_000),       # sw_power_cap
+                 (11.5, 800, 0x40, 100_000)]       # after: thermal, not counted
+    info = smp.stop()
+    assert info["samples"] == 2 and info["samples_in_process"] == 2
+    assert info["sm_mhz"] == pytest.approx((1965 + 1900) / 2)
+    assert info["sm_mhz_min"] == 1900 and info["power_w_max"] == 980.0
+    assert info["reasons"] == ["sw_power_cap"]
+    smp.local = [(9.0, 1965, 0, 1), (12.0, 1965, 0, 1)]
+    assert smp.stop()["error"] == "no samples in the timed region"
 
 
 def test_cli_rejects_short_warmup():
