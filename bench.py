@@ -17,8 +17,10 @@ reset, both outside the timed region.
 
 `value` is effective HBM GB/s: the algorithmic bytes of the step (each
 kernel's compulsory reads and writes) divided by the step time measured with
-CUDA events.  Per-kernel times come from graphs of each kernel's launches as
-the step issues them (one per layer, back to back), timed the same way.
+CUDA events.  Per-kernel times come from graphs of 1, 2, 4, 8 and 16 of each
+kernel's launches as the step issues them (one per layer, back to back),
+timed the same way: the per-launch time is the slope of graph time against
+launches, which leaves out the fixed cost of timing a graph between events.
 `--impl reference` times the CPU oracle on a bounded sample of the same step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
